@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE expert-parallel dispatch / combine hot path on B200.
+
+One step = the whole path over one batch of the workload: routing layout,
+dispatch (FP8 with the prefill workload), combine, combine backward and
+dispatch backward, all through the C ABI (libep_b200.so).  Inputs are
+seeded synthetic draws (combine_ep_get_histogram_b200.workloads) resident in
+HBM; every tensor of the prefill workload is larger than the 126 MB L2, so
+no flush is needed between steps.
+
+Prints one JSON line (rank 0).  value = effective GB/s of the step over all
+ranks (algorithmic bytes read + written by the five calls / device time);
+per-call microseconds and GB/s are in "per_call".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle on a bounded sample of the same
+workload (rank 0 only).  With N > 1 (torchrun) every rank runs an
+independent replica on its own GPU ("replicas only": the virtual-rank path
+has no inter-GPU exchange); the step time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch/combine µs/call & effective GB/s vs B200 roofline, 1 GPU"
+CALLS = ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def call_bytes(w) -> dict:
+    """Algorithmic bytes read + written per call."""
+    T, H, k, R = w.T, w.H, w.k, w.R
+    disp = T * H * 2 + (T * k * (H + 4 * (H // 128)) if w.use_fp8 else T * k * H * 2)
+    return {
+        "layout": T * k * 8 + T * R + 2 * T * k * 4,
+        "dispatch": disp,
+        "combine": T * k * H * 2 + T * k * 4 + T * H * 2,
+        "combine_backward": T * H * 2 + 2 * T * k * H * 2 + 2 * T * k * 4,
+        "dispatch_backward": T * k * H * 2 + T * H * 2,
+    }
+
+
+def peaks() -> tuple[float, str]:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons, kept only inside
+    the timed window."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.sel = []
+        try:
+            self.sel = ["-i", "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)]
+        except Exception:
+            pass
+        self.proc = None
+        self.path = None
+        self.window = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-lms", "50"] + self.sel, stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.out.close()
+        import datetime
+        sm, smax, reasons, n = [], [], set(), 0
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                if self.window and not (self.window[0] - 0.05 <= ts <= self.window[1] + 0.05):
+                    continue
+                n += 1
+                try:
+                    sm.append(float(parts[1].split()[0]))
+                    smax.append(float(parts[2].split()[0]))
+                except ValueError:
+                    pass
+                for name, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ------------------------------------------------------------- GPU arm
+
+class Path:
+    """Device buffers of one workload and one step through the C ABI."""
+
+    def __init__(self, w, d, dev):
+        import numpy as np
+        import torch
+        import combine_ep_get_histogram_b200 as ep
+        self.ep, self.w, self.dev = ep, w, dev
+        P = w.T * w.k
+
+        def bf16(a):
+            return torch.from_numpy(a.view(np.int16))
+
+        self.host = {"topk_idx": torch.from_numpy(d["topk_idx"]), "topk_weights": torch.from_numpy(d["topk_weights"]),
+                     "x": bf16(d["x"]), "y": bf16(d["y"]), "g": bf16(d["g"])}
+        self.inp = {n: t.to(dev) for n, t in self.host.items()}
+        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8)
+        self.handle = ep.Handle(self.shape, dev)
+        self.ws = ep.workspace(self.shape, dev)
+        self.recv_x = torch.empty((P, w.H), dtype=torch.uint8 if w.use_fp8 else torch.int16, device=dev)
+        self.recv_scale = torch.empty((P, w.G), dtype=torch.float32, device=dev) if w.use_fp8 else None
+        self.recv_weight = torch.empty(P, dtype=torch.float32, device=dev)
+        self.out = torch.empty((w.T, w.H), dtype=torch.int16, device=dev)
+        self.grad_y = torch.empty((P, w.H), dtype=torch.int16, device=dev)
+        self.grad_w = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
+        self.grad_x = torch.empty((w.T, w.H), dtype=torch.int16, device=dev)
+
+    def step(self, marks=None):
+        ep, i = self.ep, self.inp
+        rec = (lambda n: marks[n].record()) if marks is not None else (lambda n: None)
+        rec(0)
+        ep.ep_get_dispatch_layout(self.shape, i["topk_idx"], self.handle, self.ws)
+        rec(1)
+        ep.ep_dispatch(self.shape, i["x"], i["topk_weights"], self.handle, self.recv_x, self.recv_scale,
+                       self.recv_weight)
+        rec(2)
+        ep.ep_combine(self.shape, i["y"], i["topk_weights"], self.handle, self.out)
+        rec(3)
+        ep.ep_combine_backward(self.shape, i["g"], i["y"], i["topk_weights"], self.handle, self.grad_y,
+                               self.grad_w)
+        rec(4)
+        ep.ep_dispatch_backward(self.shape, self.grad_y, self.handle, self.grad_x)
+        rec(5)
+
+
+KERNELS_PER_STEP = 3 + 1 + 1 + 1 + 1  # layout (count, scan, assign), dispatch, combine, two backward
+
+
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from combine_ep_get_histogram_b200 import workloads as wl
+
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    w = wl.CONFIGS[args.workload]
+    d = wl.make_inputs(w, parts=("routing", "x", "y", "g"))
+    path = Path(w, d, dev)
+    stream = torch.cuda.current_stream()
+    nb = call_bytes(w)
+    step_bytes = sum(nb.values())
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        path.step()
+    barrier()
+
+    # device-timed region: K steps, per-call events on the launching stream
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    t0 = time.time()
+    for s in range(args.steps):
+        path.step(marks[s])
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    sampler.mark(t0, t1)
+    clocks = sampler.stop()
+    per_call_ms = {c: [] for c in CALLS}
+    for m in marks:
+        for ci, c in enumerate(CALLS):
+            per_call_ms[c].append(m[ci].elapsed_time(m[ci + 1]))
+    total_ms = marks[0][0].elapsed_time(marks[-1][5])
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the same C ABI: pinned host inputs in, results out, per step
+    e2e = None
+    if not args.no_e2e:
+        pin = {n: t.pin_memory() for n, t in path.host.items()}
+        outs = {"out": torch.empty_like(path.out, device="cpu").pin_memory(),
+                "grad_x": torch.empty_like(path.grad_x, device="cpu").pin_memory(),
+                "grad_w": torch.empty_like(path.grad_w, device="cpu").pin_memory()}
+        h2d = sum(t.numel() * t.element_size() for t in pin.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+        def e2e_step():
+            for n, t in pin.items():
+                path.inp[n].copy_(t, non_blocking=True)
+            path.step()
+            outs["out"].copy_(path.out, non_blocking=True)
+            outs["grad_x"].copy_(path.grad_x, non_blocking=True)
+            outs["grad_w"].copy_(path.grad_w, non_blocking=True)
+
+        for _ in range(max(1, min(args.warmup, 3))):
+            e2e_step()
+        barrier()
+        n_e2e = max(1, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": round(world * step_bytes * n_e2e / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "ms_per_step": round(e_ms / n_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank != 0:
+        return None
+
+    peak, peak_kind = peaks()
+    per_call = {}
+    for c in CALLS:
+        us = 1e3 * statistics.mean(per_call_ms[c])
+        per_call[c] = {"us": round(us, 2), "us_median": round(1e3 * statistics.median(per_call_ms[c]), 2),
+                       "bytes": nb[c], "GB_s": round(nb[c] / (us * 1e-6) / 1e9, 1),
+                       "frac_of_peak": round(nb[c] / (us * 1e-6) / 1e9 / peak, 3)}
+    dominant = max((c for c in CALLS), key=lambda c: per_call[c]["us"])
+    kernel_of = {"dispatch": "dispatch_kernel<FP8>" if w.use_fp8 else "dispatch_kernel<BF16>",
+                 "combine": "gather_reduce_kernel<weighted>", "combine_backward": "combine_backward_kernel<8>",
+                 "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel"}
+    ach = per_call[dominant]["GB_s"]
+    line = {
+        "metric": METRIC,
+        "value": round(world * step_bytes * args.steps / (total_ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8-e4m3 dispatch / bf16 combine, fp32 math" if w.use_fp8 else "bf16, fp32 math",
+        "data": "synthetic (seeded group-limited routing, N(0,1) activations)",
+        "config": {"workload": f"{w.name}: T={w.T} ({w.R} virtual ranks x {w.T // w.R} tokens), H={w.H}, "
+                               f"E={w.E}, k={w.k}, top-{w.topk_groups} of {w.n_groups} groups, "
+                               f"{'FP8' if w.use_fp8 else 'BF16'} dispatch + BF16 combine + both backward passes",
+                   "T": w.T, "H": w.H, "k": w.k, "E": w.E, "R": w.R, "use_fp8": w.use_fp8,
+                   "step_bytes": step_bytes, "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, virtual ranks"},
+        "per_call": per_call,
+        "roofline": {"kernel": kernel_of[dominant], "call": dominant, "bound": "hbm", "achieved": ach,
+                     "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 3),
+                     "peak_source": f"{peak_kind} hbm_gbs",
+                     "bytes_per_launch": nb[dominant], "traffic": None},
+        "clocks": clocks,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "e2e": e2e,
+    }
+    return line
+
+
+# -------------------------------------------------------- CPU oracle arm
+
+def oracle_pass(w, d):
+    import oracle
+    lay = oracle.layout(d["topk_idx"], w.E, w.R)
+    slots = lay["slot_of_pair"]
+    oracle.dispatch(d["x"], d["topk_weights"], slots, w.use_fp8)
+    oracle.combine(d["y"], d["topk_weights"], slots)
+    gy, _ = oracle.combine_backward(d["g"], d["y"], d["topk_weights"], slots)
+    oracle.dispatch_backward(gy, slots, w.T, w.k)
+
+
+def cpu_sample(workload: str, tokens_per_rank: int):
+    from combine_ep_get_histogram_b200 import workloads as wl
+    w = wl.CONFIGS[workload]
+    ws = w.with_(T=w.R * tokens_per_rank)
+    d = wl.make_inputs(ws, parts=("routing", "x", "y", "g"))
+    desc = (f"{w.name} shape (H={w.H}, E={w.E}, k={w.k}, R={w.R}) with T={ws.T} "
+            f"({tokens_per_rank} tokens per rank) instead of {w.T}; one full pass of the five calls")
+    return ws, d, desc
+
+
+def run_cpu_baseline(args) -> dict:
+    ws, d, desc = cpu_sample(args.workload, args.cpu_tokens_per_rank)
+    t = time.perf_counter()
+    oracle_pass(ws, d)
+    dt = time.perf_counter() - t
+    gbs = sum(call_bytes(ws).values()) / dt / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args) -> dict:
+    ws, d, desc = cpu_sample(args.workload, args.ref_tokens_per_rank)
+    for _ in range(args.warmup):
+        oracle_pass(ws, d)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_pass(ws, d)
+    dt = (time.perf_counter() - t) / args.steps
+    gbs = sum(call_bytes(ws).values()) / dt / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 dispatch / bf16 combine, fp32 math" if ws.use_fp8 else "bf16, fp32 math",
+        "data": "synthetic (seeded)", "config": {"workload": desc},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens-per-rank", type=int, default=512)
+    ap.add_argument("--ref-tokens-per-rank", type=int, default=64)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device(f"cuda:{local}"))
+    try:
+        line = run_ours(args, rank, world, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = run_cpu_baseline(args)
+            else:
+                line["cpu_baseline"] = None
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,76 @@
+// Device helpers shared by the layout and data-movement kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ep {
+
+constexpr int kWarp = 32;
+constexpr int kMaxK = 32;
+constexpr int kMaxE = 1024;
+constexpr int kMaxR = 256;
+constexpr int kGroup = 128;                   // channels per FP8 scale
+constexpr int kLaneElems = 16;                // channels a lane moves per chunk
+constexpr int kChunk = kWarp * kLaneElems;    // 512 channels per warp chunk
+constexpr int kLanesPerGroup = kGroup / kLaneElems;  // 8
+constexpr int kTilePairs = 1024;              // layout tile: pairs per CTA
+constexpr int kTileFlagBytes = 32768;         // layout tile: tokens x ranks flag bytes
+constexpr int kLayoutThreads = 256;
+constexpr int kLayoutWarps = kLayoutThreads / kWarp;
+constexpr int kMaxChunksPerWarp = (kTilePairs / kLayoutWarps + kWarp - 1) / kWarp;  // 4
+constexpr float kE4M3Max = 448.0f;
+
+// 16-byte load of data that no thread writes during the kernel: non-coherent
+// path, no L1 allocation, 256-byte L2 prefetch (the aggressive load the pages
+// describe, used only on read-only inputs).
+__device__ __forceinline__ uint4 ld_ro_v4(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+  *reinterpret_cast<uint4*>(p) = v;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Two fp32 values -> packed bf16x2 (round to nearest even); `lo` lands in the
+// low half, which is the lower address in memory.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 values -> packed E4M3 codes (round to nearest even, saturating to
+// +-448); `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+  f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+  f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+  f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float* f) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                    pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+}  // namespace ep

@@ -1,0 +1,349 @@
+// C ABI of libep_b200.so (declared in include/ep.h): argument checks on the
+// host, launch configuration, status codes.  Every step of the hot path runs
+// in the kernels of layout.cuh and movement.cuh; nothing here touches data.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "ep.h"
+#include "layout.cuh"
+#include "movement.cuh"
+
+namespace {
+
+using namespace ep;
+
+thread_local char g_last_cuda_error[256] = "";
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return EP_OK;
+  std::snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+                cudaGetErrorString(e));
+  return EP_ERR_CUDA;
+}
+
+bool debug_mode() {
+  static const bool on = [] {
+    const char* s = std::getenv("EP_DEBUG");
+    return s != nullptr && s[0] == '1';
+  }();
+  return on;
+}
+
+// Per-device facts, read once.
+struct DeviceInfo {
+  int sms = 0;
+  bool supported = false;
+  int occ_count = 0, occ_scan = 0, occ_assign = 0;
+  int occ_disp_bf16 = 0, occ_disp_fp8 = 0, occ_comb = 0, occ_dbwd = 0, occ_cbwd8 = 0, occ_cbwd32 = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+bool g_dev_ready[kMaxDevices] = {};
+
+int occupancy(const void* fn, int threads, size_t smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess) return 1;
+  return n > 0 ? n : 1;
+}
+
+int device_info(const DeviceInfo** out) {
+  int dev = 0;
+  int st = cuda_status(cudaGetDevice(&dev));
+  if (st != EP_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return EP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  if (!g_dev_ready[dev]) {
+    DeviceInfo d;
+    cudaDeviceProp prop;
+    st = cuda_status(cudaGetDeviceProperties(&prop, dev));
+    if (st != EP_OK) return st;
+    d.sms = prop.multiProcessorCount;
+    d.supported = prop.major == 10 && prop.minor == 0;
+    if (d.supported) {
+      d.occ_count = occupancy(reinterpret_cast<const void*>(layout_count_kernel), kLayoutThreads,
+                              (kMaxE + kMaxR) * 4 + kTileFlagBytes);
+      d.occ_disp_bf16 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<false>), kMoveThreads, 0);
+      d.occ_disp_fp8 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<true>), kMoveThreads, 0);
+      d.occ_comb = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<true>), kMoveThreads, 0);
+      d.occ_dbwd = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false>), kMoveThreads, 0);
+      d.occ_cbwd8 = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<8>), kMoveThreads, 0);
+      d.occ_cbwd32 =
+          occupancy(reinterpret_cast<const void*>(combine_backward_kernel<kMaxK>), kMoveThreads, 0);
+      cudaGetLastError();
+    }
+    g_dev[dev] = d;
+    g_dev_ready[dev] = true;
+  }
+  if (!g_dev[dev].supported) return EP_ERR_UNSUPPORTED;
+  *out = &g_dev[dev];
+  return EP_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(const ep_shape_t* s) {
+  if (s == nullptr) return EP_ERR_INVALID_ARG;
+  if (s->T < 0 || s->k < 1 || s->k > kMaxK || s->E < 1 || s->E > kMaxE || s->R < 1 ||
+      s->R > kMaxR || s->R > s->E || s->E % s->R != 0 || s->T % s->R != 0)
+    return EP_ERR_INVALID_ARG;
+  if (s->H < 8 || s->H % 8 != 0) return EP_ERR_INVALID_ARG;
+  if (s->use_fp8 != 0 && s->use_fp8 != 1) return EP_ERR_INVALID_ARG;
+  if (s->use_fp8 && s->H % kGroup != 0) return EP_ERR_INVALID_ARG;
+  if (s->num_sms < 0) return EP_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s->T) * s->k > 0x7fffffffLL) return EP_ERR_INVALID_ARG;
+  return EP_OK;
+}
+
+int check_handle(const ep_shape_t* s, const ep_handle_t* h) {
+  if (h == nullptr) return EP_ERR_INVALID_ARG;
+  const void* arrays[] = {h->num_tokens_per_expert, h->expert_offset, h->num_tokens_per_rank,
+                          h->count_src_rank_expert, h->src_rank_expert_offset, h->slot_of_pair,
+                          h->src_of_slot, h->error_word};
+  for (const void* a : arrays)
+    if (a == nullptr || !aligned(a, 4)) return EP_ERR_INVALID_ARG;
+  if (h->is_token_in_rank == nullptr && s->T > 0) return EP_ERR_INVALID_ARG;
+  return EP_OK;
+}
+
+// Row arrays must be non-null (when they hold data) and 16-byte aligned.
+bool rows_ok(const void* p, int64_t rows) { return rows == 0 || (p != nullptr && aligned(p, 16)); }
+bool f32_ok(const void* p, int64_t n) { return n == 0 || (p != nullptr && aligned(p, 4)); }
+
+int grid_cap(const DeviceInfo& d, const ep_shape_t* s, int occ) {
+  const int sms = (s->num_sms > 0 && s->num_sms < d.sms) ? s->num_sms : d.sms;
+  return sms * occ;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct LayoutGeometry {
+  int tile_t, tiles_per_rank, nt, ncol;
+  size_t colhist_bytes, coltotal_bytes, total_bytes;
+};
+
+LayoutGeometry layout_geometry(const ep_shape_t* s) {
+  LayoutGeometry g;
+  const int Tr = s->T / s->R;
+  g.tile_t = kTilePairs / s->k;
+  if (g.tile_t > kTileFlagBytes / s->R) g.tile_t = kTileFlagBytes / s->R;
+  if (g.tile_t < 1) g.tile_t = 1;
+  g.tiles_per_rank = static_cast<int>(ceil_div(Tr, g.tile_t));
+  g.nt = s->R * g.tiles_per_rank;
+  g.ncol = s->E + s->R;
+  auto round256 = [](size_t b) { return (b + 255) / 256 * 256; };
+  g.colhist_bytes = round256(static_cast<size_t>(g.ncol) * g.nt * 4);
+  g.coltotal_bytes = round256(static_cast<size_t>(g.ncol) * 4);
+  g.total_bytes = g.colhist_bytes + g.coltotal_bytes;
+  return g;
+}
+
+MoveParams move_params(const ep_shape_t* s, const ep_handle_t* h, const float* w) {
+  MoveParams p;
+  p.T = s->T;
+  p.H = s->H;
+  p.k = s->k;
+  p.G = s->H / kGroup;
+  p.chunks = static_cast<int>(ceil_div(s->H, kChunk));
+  p.slot_of_pair = h->slot_of_pair;
+  p.topk_weights = w;
+  return p;
+}
+
+int finish(const ep_handle_t* h, cudaStream_t stream) {
+  int st = cuda_status(cudaGetLastError());
+  if (st != EP_OK || !debug_mode()) return st;
+  return ep_get_error(h, reinterpret_cast<ep_stream_t>(stream));
+}
+
+int movement_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t units_per_warp_grid) {
+  const int64_t need = ceil_div(units_per_warp_grid, kMoveWarps);
+  const int64_t cap = grid_cap(d, s, occ);
+  return static_cast<int>(need < cap ? need : cap);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ep_handle_sizes(const ep_shape_t* shape, int64_t counts[9]) {
+  int st = check_shape(shape);
+  if (st != EP_OK || counts == nullptr) return EP_ERR_INVALID_ARG;
+  const int64_t T = shape->T, k = shape->k, E = shape->E, R = shape->R;
+  const int64_t c[9] = {E, E + 1, R, R * E, R * E, T * R, T * k, T * k, 1};
+  for (int i = 0; i < 9; ++i) counts[i] = c[i];
+  return EP_OK;
+}
+
+size_t ep_workspace_size(const ep_shape_t* shape) {
+  if (check_shape(shape) != EP_OK) return 0;
+  return layout_geometry(shape).total_bytes;
+}
+
+int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, const ep_handle_t* handle,
+                           void* workspace, size_t workspace_bytes, ep_stream_t stream) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  const LayoutGeometry g = layout_geometry(shape);
+  if (shape->T > 0 && (topk_idx == nullptr || !aligned(topk_idx, 8))) return EP_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < g.total_bytes)
+    return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+
+  LayoutParams p;
+  p.topk_idx = topk_idx;
+  p.T = shape->T;
+  p.k = shape->k;
+  p.E = shape->E;
+  p.R = shape->R;
+  p.Tr = shape->T / shape->R;
+  p.Er = shape->E / shape->R;
+  p.tile_t = g.tile_t;
+  p.tiles_per_rank = g.tiles_per_rank;
+  p.nt = g.nt;
+  p.ncol = g.ncol;
+  p.colhist = static_cast<int32_t*>(workspace);
+  p.coltotal = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + g.colhist_bytes);
+  p.num_tokens_per_expert = handle->num_tokens_per_expert;
+  p.expert_offset = handle->expert_offset;
+  p.num_tokens_per_rank = handle->num_tokens_per_rank;
+  p.count_src_rank_expert = handle->count_src_rank_expert;
+  p.src_rank_expert_offset = handle->src_rank_expert_offset;
+  p.is_token_in_rank = handle->is_token_in_rank;
+  p.slot_of_pair = handle->slot_of_pair;
+  p.src_of_slot = handle->src_of_slot;
+  p.error_word = handle->error_word;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (g.nt > 0) {
+    const size_t smem = static_cast<size_t>(g.ncol) * 4 + static_cast<size_t>(g.tile_t) * shape->R;
+    layout_count_kernel<<<g.nt, kLayoutThreads, smem, s>>>(p);
+  }
+  layout_scan_kernel<<<g.ncol, kLayoutThreads, 0, s>>>(p);
+  const size_t smem_assign = static_cast<size_t>(shape->E + 1 + kLayoutWarps * shape->E) * 4;
+  layout_assign_kernel<<<g.nt > 0 ? g.nt : 1, kLayoutThreads, smem_assign, s>>>(p);
+  return finish(handle, s);
+}
+
+int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weights, const ep_handle_t* handle,
+                void* recv_x, float* recv_scale, float* recv_weight, ep_stream_t stream) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  const int64_t T = shape->T, P = T * shape->k;
+  if (!rows_ok(x, T) || !rows_ok(recv_x, P) || !f32_ok(topk_weights, P)) return EP_ERR_INVALID_ARG;
+  if (shape->use_fp8 && !f32_ok(recv_scale, P)) return EP_ERR_INVALID_ARG;
+  if (recv_weight != nullptr && !aligned(recv_weight, 4)) return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  const MoveParams p = move_params(shape, handle, topk_weights);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t units = T * p.chunks;
+  if (shape->use_fp8) {
+    dispatch_kernel<true><<<movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s>>>(
+        p, static_cast<const uint16_t*>(x), recv_x, recv_scale, recv_weight);
+  } else {
+    dispatch_kernel<false><<<movement_grid(*d, shape, d->occ_disp_bf16, units), kMoveThreads, 0, s>>>(
+        p, static_cast<const uint16_t*>(x), recv_x, nullptr, recv_weight);
+  }
+  return finish(handle, s);
+}
+
+int ep_combine(const ep_shape_t* shape, const void* y, const float* topk_weights, const ep_handle_t* handle,
+               void* out, ep_stream_t stream) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  const int64_t T = shape->T, P = T * shape->k;
+  if (!rows_ok(y, P) || !rows_ok(out, T) || !f32_ok(topk_weights, P)) return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  const MoveParams p = move_params(shape, handle, topk_weights);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  gather_reduce_kernel<true><<<movement_grid(*d, shape, d->occ_comb, T * p.chunks), kMoveThreads, 0, s>>>(
+      p, static_cast<const uint16_t*>(y), static_cast<uint16_t*>(out));
+  return finish(handle, s);
+}
+
+int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const void* y,
+                        const float* topk_weights, const ep_handle_t* handle, void* grad_y, float* grad_w,
+                        ep_stream_t stream) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  const int64_t T = shape->T, P = T * shape->k;
+  if (!rows_ok(grad_out, T) || !rows_ok(y, P) || !rows_ok(grad_y, P) || !f32_ok(topk_weights, P) ||
+      !f32_ok(grad_w, P))
+    return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  const MoveParams p = move_params(shape, handle, topk_weights);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool small_k = shape->k <= 8;
+  const int64_t cap = grid_cap(*d, shape, small_k ? d->occ_cbwd8 : d->occ_cbwd32);
+  const int grid = static_cast<int>(T < cap ? T : cap);
+  if (small_k)
+    combine_backward_kernel<8><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_out),
+                                                             static_cast<const uint16_t*>(y),
+                                                             static_cast<uint16_t*>(grad_y), grad_w);
+  else
+    combine_backward_kernel<kMaxK><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_out),
+                                                                 static_cast<const uint16_t*>(y),
+                                                                 static_cast<uint16_t*>(grad_y), grad_w);
+  return finish(handle, s);
+}
+
+int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv, const ep_handle_t* handle,
+                         void* grad_x, ep_stream_t stream) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  const int64_t T = shape->T, P = T * shape->k;
+  if (!rows_ok(grad_recv, P) || !rows_ok(grad_x, T)) return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  const MoveParams p = move_params(shape, handle, nullptr);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  gather_reduce_kernel<false><<<movement_grid(*d, shape, d->occ_dbwd, T * p.chunks), kMoveThreads, 0, s>>>(
+      p, static_cast<const uint16_t*>(grad_recv), static_cast<uint16_t*>(grad_x));
+  return finish(handle, s);
+}
+
+int ep_get_error(const ep_handle_t* handle, ep_stream_t stream) {
+  if (handle == nullptr || handle->error_word == nullptr) return EP_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  int st = cuda_status(cudaStreamSynchronize(s));
+  if (st != EP_OK) return st;
+  if ((st = cuda_status(cudaMemcpyAsync(&word, handle->error_word, 4, cudaMemcpyDeviceToHost, s))) != EP_OK)
+    return st;
+  if ((st = cuda_status(cudaMemsetAsync(handle->error_word, 0, 4, s))) != EP_OK) return st;
+  if ((st = cuda_status(cudaStreamSynchronize(s))) != EP_OK) return st;
+  return (word & 1) ? EP_ERR_BAD_INDEX : EP_OK;
+}
+
+const char* ep_status_string(int status) {
+  switch (status) {
+    case EP_OK: return "EP_OK";
+    case EP_ERR_INVALID_ARG: return "EP_ERR_INVALID_ARG: null or misaligned pointer, or shape outside the limits";
+    case EP_ERR_BAD_INDEX: return "EP_ERR_BAD_INDEX: a topk_idx entry outside [-1, E)";
+    case EP_ERR_CUDA: return "EP_ERR_CUDA: a CUDA call or kernel launch failed";
+    case EP_ERR_UNSUPPORTED: return "EP_ERR_UNSUPPORTED: the current device is not an sm_100 GPU";
+    default: return "unknown ep status";
+  }
+}
+
+const char* ep_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

@@ -1,0 +1,158 @@
+/*
+ * ep.h — C ABI of the B200 (sm_100a) MoE expert-parallel dispatch / combine
+ * library, libep_b200.so.
+ *
+ * What the operations are (the pages describe them in words, without
+ * formulas; citations are page title + section):
+ *  - dispatch sends every token to the k experts its router picked and
+ *    returns the received tokens, their gate weights and a handle; combine
+ *    brings the experts' outputs back to each token's rank and sums them
+ *    using that handle; the same handle serves combine_backward and
+ *    dispatch_backward ("DeepEP：MoE 专家并行 EP 通信 kernel 编译与使用指南",
+ *    zhouruolin.cn, section 五 使用方法 and FAQ Q5).
+ *  - FP8 dispatch with BF16 combine is the standard precision pair
+ *    (blog.hotdry.top "deepep-expert-parallel-communication-library",
+ *    section 五 实践建议; czhn.yksolo.com "DeepSeek 开源周第二弹": 原生 FP8
+ *    调度支持), and the precision conversion is fused into the data movement
+ *    ("DeepEP：专为MoE模型打造的All-to-All通信库", bjdmk.com.cn, section 3.2).
+ *  - the per-expert token counts are the quantity one inspects for load skew
+ *    (bjdmk.com.cn, section 5.2).
+ *  - the number of SMs a call may use is a caller knob (blog.hotdry.top,
+ *    section 二 SM 资源控制).
+ *
+ * Model of the expert-parallel world: one GPU, R virtual ranks.  Rank r owns
+ * source tokens [r*T/R, (r+1)*T/R) and experts [r*E/R, (r+1)*E/R).  Every
+ * receive buffer is one array of P = T*k rows in expert-major order; rank r's
+ * partition is rows [expert_offset[r*E/R], expert_offset[(r+1)*E/R]).
+ *
+ * Numerics (the pages do not fix them; these are the definitions used):
+ *  - slots: the pairs routed to expert e take rows [expert_offset[e],
+ *    expert_offset[e+1]) in increasing (token t, top-k position j) order,
+ *    i.e. (source rank, source token) order.  topk_idx = -1 masks a pair.
+ *  - FP8 (OCP E4M3, largest finite 448): per token and 128-channel group,
+ *    amax = max |x| (fp32), scale = amax / 448 (fp32 IEEE division; 1.0 if
+ *    that is 0), code = E4M3(x / scale) with IEEE fp32 division, round to
+ *    nearest even, saturating to +-448.
+ *  - combine: acc = +0.0f; acc = fmaf(w[t,j], y[slot(t,j)], acc) for
+ *    j = 0..k-1 in order (masked pairs skipped); out = bf16 RNE(acc).
+ *  - combine_backward: grad_y[slot(t,j)] = bf16 RNE(w[t,j] * g[t]) (one fp32
+ *    product); grad_w[t,j] = sum_h g[t,h] * y[slot(t,j),h] in fp32 (the
+ *    summation order is the kernel's).
+ *  - dispatch_backward: grad_x[t] = bf16 RNE(sum_j grad_recv[slot(t,j)]),
+ *    fp32 adds from +0.0f in j order (straight-through for FP8).
+ *
+ * Conventions shared by every entry point:
+ *  - All array arguments are DEVICE pointers owned by the caller, except the
+ *    ep_shape_t / ep_handle_t structs themselves, which are read from host
+ *    memory during the call only.  The library never allocates, never frees
+ *    and never synchronises the stream (except ep_get_error, and every call
+ *    when the environment variable EP_DEBUG=1 is set).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Calls on one handle must not overlap; results are defined
+ *    once the stream reaches them.
+ *  - bf16 arrays are uint16 bit patterns; rows of bf16 / fp8 arrays must start
+ *    on 16-byte boundaries (H % 8 == 0 and 16-byte aligned base pointers).
+ *  - Return value: EP_OK or an ep_status_t code.  Argument errors are found
+ *    on the host before anything is enqueued.  Out-of-range expert ids are
+ *    found on the device: the pair is treated as masked and bit 0 of
+ *    handle->error_word is set; ep_get_error reports it.
+ *  - Limits: 0 <= T, T % R == 0, 1 <= k <= 32, 1 <= E <= 1024, 1 <= R <= E,
+ *    E % R == 0, T*k < 2^31, 8 <= H, H % 8 == 0 (H % 128 == 0 with FP8).
+ */
+#ifndef EP_B200_H
+#define EP_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* ep_stream_t;
+
+typedef enum {
+  EP_OK = 0,
+  EP_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, shape outside the limits */
+  EP_ERR_BAD_INDEX = 2,    /* a topk_idx entry outside [-1, E) (from ep_get_error) */
+  EP_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+  EP_ERR_UNSUPPORTED = 4   /* the current device is not an sm_100 GPU */
+} ep_status_t;
+
+/* Problem shape. T tokens over R virtual ranks, hidden H, top-k, E experts. */
+typedef struct {
+  int32_t T, H, k, E, R;
+  int32_t use_fp8; /* 1: dispatch writes E4M3 codes + fp32 scales; 0: bf16 rows */
+  int32_t num_sms; /* SMs a call may fill: 0 = all.  Caps each grid at
+                      num_sms x (resident CTAs per SM). */
+} ep_shape_t;
+
+/* The dispatch handle: device arrays written by ep_get_dispatch_layout and
+ * read by the other calls.  Sizes are given by ep_handle_sizes. */
+typedef struct {
+  int32_t* num_tokens_per_expert;  /* [E]   pairs routed to each expert */
+  int32_t* expert_offset;          /* [E+1] exclusive prefix sum of the above */
+  int32_t* num_tokens_per_rank;    /* [R]   tokens with >= 1 pair on rank r */
+  int32_t* count_src_rank_expert;  /* [R*E] pairs from source rank r to expert e */
+  int32_t* src_rank_expert_offset; /* [R*E] first row of (source rank r, expert e) */
+  uint8_t* is_token_in_rank;       /* [T*R] 1 if token t has a pair on rank r */
+  int32_t* slot_of_pair;           /* [T*k] receive row of pair (t,j); -1 if masked */
+  int32_t* src_of_slot;            /* [T*k] t*k+j of the pair in each row; -1 past the last row */
+  int32_t* error_word;             /* [1]   device error bits; must be 0 before first use */
+} ep_handle_t;
+
+/* Element counts of each handle array, in struct order (9 entries). */
+int ep_handle_sizes(const ep_shape_t* shape, int64_t counts[9]);
+
+/* Bytes of device scratch ep_get_dispatch_layout needs (a multiple of 256). */
+size_t ep_workspace_size(const ep_shape_t* shape);
+
+/* Routing layout: per-expert and per-rank histograms, offsets,
+ * is_token_in_rank and the slot of every (token, expert) pair.
+ * topk_idx: [T,k] int64 row-major, device.  workspace: device scratch of at
+ * least ep_workspace_size bytes, 256-byte aligned, contents irrelevant.
+ * Three kernels: tile histograms, column scans, slot assignment. */
+int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx,
+                           const ep_handle_t* handle, void* workspace,
+                           size_t workspace_bytes, ep_stream_t stream);
+
+/* Dispatch: x [T,H] bf16 -> recv_x [P,H] (bf16, or E4M3 codes when
+ * use_fp8), recv_scale [P,H/128] fp32 (required with use_fp8, else ignored),
+ * recv_weight [P] fp32 = topk_weights of each row's pair (may be NULL).
+ * topk_weights [T,k] fp32.  Rows past expert_offset[E] are not written. */
+int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weights,
+                const ep_handle_t* handle, void* recv_x, float* recv_scale,
+                float* recv_weight, ep_stream_t stream);
+
+/* Combine: y [P,H] bf16 (expert outputs in receive order), topk_weights
+ * [T,k] fp32 -> out [T,H] bf16.  A token with no valid pair gets +0. */
+int ep_combine(const ep_shape_t* shape, const void* y, const float* topk_weights,
+               const ep_handle_t* handle, void* out, ep_stream_t stream);
+
+/* Backward of combine: grad_out [T,H] bf16, y [P,H] bf16, topk_weights [T,k]
+ * -> grad_y [P,H] bf16 (rows of masked pairs untouched), grad_w [T,k] fp32
+ * (0 for masked pairs). */
+int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const void* y,
+                        const float* topk_weights, const ep_handle_t* handle,
+                        void* grad_y, float* grad_w, ep_stream_t stream);
+
+/* Backward of dispatch: grad_recv [P,H] bf16 -> grad_x [T,H] bf16. */
+int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv,
+                         const ep_handle_t* handle, void* grad_x, ep_stream_t stream);
+
+/* Synchronises `stream`, reads handle->error_word, clears it, and returns
+ * EP_ERR_BAD_INDEX if a bad expert id was seen since the last call, EP_OK if
+ * not, EP_ERR_CUDA if the stream reports an error. */
+int ep_get_error(const ep_handle_t* handle, ep_stream_t stream);
+
+/* Static description of a status code. */
+const char* ep_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread ("" if none). */
+const char* ep_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EP_B200_H */

@@ -1,0 +1,126 @@
+"""Helpers for the GPU parity tests: run the CUDA path through the C ABI on
+numpy inputs, and compare with the CPU oracle."""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import combine_ep_get_histogram_b200 as ep
+
+LAYOUT_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank",
+                 "count_src_rank_expert", "src_rank_expert_offset", "is_token_in_rank",
+                 "slot_of_pair", "src_of_slot")
+
+
+def to_dev(a: np.ndarray, device) -> torch.Tensor:
+    if a.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def bf16_host(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+class GpuPath:
+    """One workload on the GPU: the handle, the layout and the buffers."""
+
+    def __init__(self, w, topk_idx: np.ndarray, topk_weights: np.ndarray, device,
+                 use_fp8: bool | None = None, num_sms: int = 0):
+        self.w = w
+        self.device = device
+        self.use_fp8 = w.use_fp8 if use_fp8 is None else use_fp8
+        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, self.use_fp8, num_sms)
+        self.handle = ep.Handle(self.shape, device)
+        self.ws = ep.workspace(self.shape, device)
+        self.idx = to_dev(topk_idx, device)
+        self.wts = to_dev(topk_weights.astype(np.float32), device)
+
+    def layout(self):
+        ep.ep_get_dispatch_layout(self.shape, self.idx, self.handle, self.ws)
+        return self
+
+    def layout_host(self) -> dict:
+        torch.cuda.synchronize()
+        return {n: self.handle.tensors[n].cpu().numpy()[: self._count(n)] for n in LAYOUT_FIELDS}
+
+    def _count(self, n):
+        return ep.handle_sizes(self.shape)[n]
+
+    def dispatch(self, x_dev, fill=0):
+        w = self.w
+        P = w.T * w.k
+        if self.use_fp8:
+            recv_x = torch.full((max(P, 1), w.H), fill, dtype=torch.uint8, device=self.device)
+            recv_scale = torch.full((max(P, 1), w.H // 128), float(fill), dtype=torch.float32,
+                                    device=self.device)
+        else:
+            recv_x = torch.full((max(P, 1), w.H), fill, dtype=torch.int16, device=self.device)
+            recv_scale = None
+        recv_weight = torch.full((max(P, 1),), float(fill), dtype=torch.float32, device=self.device)
+        ep.ep_dispatch(self.shape, x_dev, self.wts, self.handle, recv_x, recv_scale, recv_weight)
+        return recv_x, recv_scale, recv_weight
+
+    def combine(self, y_dev):
+        out = torch.empty((max(self.w.T, 1), self.w.H), dtype=torch.int16, device=self.device)
+        ep.ep_combine(self.shape, y_dev, self.wts, self.handle, out)
+        return out
+
+    def combine_backward(self, g_dev, y_dev):
+        w = self.w
+        grad_y = torch.zeros((max(w.T * w.k, 1), w.H), dtype=torch.int16, device=self.device)
+        grad_w = torch.full((max(w.T, 1), w.k), -7.0, dtype=torch.float32, device=self.device)
+        ep.ep_combine_backward(self.shape, g_dev, y_dev, self.wts, self.handle, grad_y, grad_w)
+        return grad_y, grad_w
+
+    def dispatch_backward(self, grad_recv_dev):
+        grad_x = torch.empty((max(self.w.T, 1), self.w.H), dtype=torch.int16, device=self.device)
+        ep.ep_dispatch_backward(self.shape, grad_recv_dev, self.handle, grad_x)
+        return grad_x
+
+
+def assert_layout_equal(got: dict, ref: dict):
+    for n in LAYOUT_FIELDS:
+        a = np.asarray(got[n]).astype(np.int64)
+        b = np.asarray(ref[n]).astype(np.int64)
+        assert a.shape == b.shape, n
+        if not np.array_equal(a, b):
+            bad = np.nonzero(a != b)[0]
+            raise AssertionError(f"{n}: {bad.size} mismatches, first at {bad[:5]}: "
+                                 f"gpu {a[bad[:5]]} oracle {b[bad[:5]]}")
+
+
+def assert_bits_equal(name, got: np.ndarray, ref: np.ndarray):
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    if not np.array_equal(got, ref):
+        bad = np.argwhere(got != ref)
+        raise AssertionError(f"{name}: {len(bad)} of {got.size} differ, first {bad[:5].tolist()}: "
+                             f"gpu {got[tuple(bad[:5].T)]} oracle {ref[tuple(bad[:5].T)]}")
+
+
+def bf16_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance in bf16 units in the last place (ordered-integer metric)."""
+    def ordered(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x8000, 0x8000 - (x & 0x7FFF), 0x8000 + x)
+    return np.abs(ordered(a) - ordered(b))
+
+
+def grad_w_close(got: np.ndarray, ref: np.ndarray, rel=1e-2):
+    """|got - ref| <= rel * |ref|, or <= rel * rms(ref) where ref is near 0."""
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2))) if ref.size else 0.0
+    err = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    ok = (err <= rel * np.abs(ref)) | (err <= rel * rms)
+    return bool(np.all(ok)), float(np.max(err / np.maximum(np.abs(ref), rms)) if ref.size else 0.0)
+
+
+def sample_tokens(T: int, R: int, n: int, seed: int = 123) -> np.ndarray:
+    """Random tokens plus the first and last token of every virtual rank."""
+    if T == 0:
+        return np.zeros(0, np.int64)
+    rng = np.random.default_rng(seed)
+    Tr = T // R
+    edges = np.concatenate([np.arange(R) * Tr, np.arange(1, R + 1) * Tr - 1])
+    pick = rng.choice(T, size=min(n, T), replace=False)
+    return np.unique(np.concatenate([edges, pick]))

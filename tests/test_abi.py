@@ -1,0 +1,114 @@
+"""The C ABI library loads, exports every entry point include/ep.h declares,
+and rejects bad arguments on the host before any CUDA call (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_ep_get_histogram_b200 as ep
+from combine_ep_get_histogram_b200 import ep as binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ep.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ep_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("ep_get_dispatch_layout", "ep_dispatch", "ep_combine", "ep_combine_backward",
+              "ep_dispatch_backward", "ep_get_error", "ep_workspace_size", "ep_handle_sizes"):
+        assert n in names
+    assert set(names) == set(binding.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for st in range(5):
+        assert binding.status_string(st).startswith("EP_")
+
+
+def test_handle_sizes_and_workspace():
+    s = ep.make_shape(T=64, H=256, k=4, E=16, R=4)
+    sizes = ep.handle_sizes(s)
+    assert sizes == {"num_tokens_per_expert": 16, "expert_offset": 17, "num_tokens_per_rank": 4,
+                     "count_src_rank_expert": 64, "src_rank_expert_offset": 64,
+                     "is_token_in_rank": 256, "slot_of_pair": 256, "src_of_slot": 256,
+                     "error_word": 1}
+    ws = ep.workspace_size(s)
+    assert ws > 0 and ws % 256 == 0
+    big = ep.make_shape(T=32768, H=7168, k=8, E=256, R=8, use_fp8=True)
+    # (E + R) columns x (8 ranks x 32 tiles of 128 tokens), plus the totals
+    assert ep.workspace_size(big) == (264 * 256 * 4 + 255) // 256 * 256 + (264 * 4 + 255) // 256 * 256
+
+
+BAD_SHAPES = [
+    dict(T=63, H=256, k=4, E=16, R=4),      # T % R
+    dict(T=64, H=256, k=4, E=18, R=4),      # E % R
+    dict(T=64, H=256, k=0, E=16, R=4),      # k < 1
+    dict(T=64, H=256, k=33, E=64, R=4),     # k > 32
+    dict(T=64, H=256, k=4, E=2048, R=4),    # E > 1024
+    dict(T=64, H=250, k=4, E=16, R=4),      # H % 8
+    dict(T=64, H=320, k=4, E=16, R=4, use_fp8=True),  # H % 128 with FP8
+    dict(T=64, H=256, k=4, E=4, R=8),       # R > E
+    dict(T=-4, H=256, k=4, E=16, R=4),
+    dict(T=64, H=256, k=4, E=16, R=4, num_sms=-1),
+]
+
+
+@pytest.mark.parametrize("kw", BAD_SHAPES)
+def test_bad_shapes_rejected_on_host(kw):
+    s = ep.make_shape(**kw)
+    lib = ep.library()
+    assert lib.ep_workspace_size(ctypes.byref(s)) == 0
+    h = binding.ep_handle_t(*([4096] * 9))
+    fake = 1 << 20  # never dereferenced: validation fails first
+    assert lib.ep_get_dispatch_layout(ctypes.byref(s), fake, ctypes.byref(h), fake, 1 << 20, None) == 1
+    assert lib.ep_dispatch(ctypes.byref(s), fake, fake, ctypes.byref(h), fake, fake, None, None) == 1
+    assert lib.ep_combine(ctypes.byref(s), fake, fake, ctypes.byref(h), fake, None) == 1
+    assert lib.ep_combine_backward(ctypes.byref(s), fake, fake, fake, ctypes.byref(h), fake, fake, None) == 1
+    assert lib.ep_dispatch_backward(ctypes.byref(s), fake, ctypes.byref(h), fake, None) == 1
+
+
+def test_bad_pointers_rejected_on_host():
+    s = ep.make_shape(T=64, H=256, k=4, E=16, R=4, use_fp8=True)
+    lib = ep.library()
+    good = 1 << 20
+    h = binding.ep_handle_t(*([good] * 9))
+    sref, href = ctypes.byref(s), ctypes.byref(h)
+    ws = ep.workspace_size(s)
+    # layout: null index, misaligned index, small / misaligned workspace, null handle array
+    assert lib.ep_get_dispatch_layout(sref, None, href, good, ws, None) == 1
+    assert lib.ep_get_dispatch_layout(sref, good + 4, href, good, ws, None) == 1
+    assert lib.ep_get_dispatch_layout(sref, good, href, good, ws - 1, None) == 1
+    assert lib.ep_get_dispatch_layout(sref, good, href, good + 16, ws, None) == 1
+    h2 = binding.ep_handle_t(*([good] * 6 + [0] + [good] * 2))
+    assert lib.ep_get_dispatch_layout(sref, good, ctypes.byref(h2), good, ws, None) == 1
+    assert lib.ep_get_dispatch_layout(sref, good, None, good, ws, None) == 1
+    # dispatch: rows must be 16-byte aligned, FP8 needs recv_scale
+    assert lib.ep_dispatch(sref, good + 8, good, href, good, good, None, None) == 1
+    assert lib.ep_dispatch(sref, good, good, href, good + 2, good, None, None) == 1
+    assert lib.ep_dispatch(sref, good, good, href, good, None, None, None) == 1
+    assert lib.ep_dispatch(sref, good, good + 2, href, good, good, None, None) == 1
+    assert lib.ep_combine(sref, good + 8, good, href, good, None) == 1
+    assert lib.ep_combine(sref, good, good, href, None, None) == 1
+    assert lib.ep_combine_backward(sref, good, good, good, href, good, None, None) == 1
+    assert lib.ep_dispatch_backward(sref, good, href, good + 4, None) == 1
+    assert lib.ep_get_error(None, None) == 1
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(binding, "_LIB", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.library()
