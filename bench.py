@@ -190,7 +190,7 @@ def run_ours(args, rank, world, local):
 
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
-    w = wl.CONFIGS[args.workload]
+    w = workload(args)
     d = wl.make_inputs(w, parts=("routing", "x", "y", "g"))
     path = Path(w, d, dev)
     stream = torch.cuda.current_stream()
@@ -312,6 +312,14 @@ def run_ours(args, rank, world, local):
     return line
 
 
+def workload(args):
+    from combine_ep_get_histogram_b200 import workloads as wl
+    w = wl.CONFIGS[args.workload]
+    if args.tokens_per_rank:
+        w = w.with_(T=w.R * args.tokens_per_rank)
+    return w
+
+
 # -------------------------------------------------------- CPU oracle arm
 
 def oracle_pass(w, d):
@@ -371,6 +379,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--tokens-per-rank", type=int, default=0,
+                    help="resize the workload to R x this many tokens (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens-per-rank", type=int, default=512)

@@ -33,6 +33,68 @@ constexpr int kMoveWarps = kMoveThreads / kWarp;
 
 // ---------------------------------------------------------------- dispatch
 
+// f[i] <- x_i / scale, rounded to nearest even in fp32, for 16 values of one
+// 128-channel group (scale >= the group's amax / 448).
+//
+// Fast path (Markstein's division with a correctly rounded reciprocal, P.
+// Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): r = RN(1/scale), q0 = RN(|x|*r),
+// e = |x| - q0*scale (exact through the FMA), q = RN(q0 + e*r), sign copied
+// back.  It gives the correctly rounded quotient unless the remainder
+// underflows; for inputs that are bf16 values this holds whenever |x| >=
+// 2^-105 and scale is a normal number with a finite reciprocal.  Every
+// (x, amax) pair of bf16 values was checked: the resulting E4M3 codes equal
+// those of the IEEE division.  Other elements (zeros excepted) take the IEEE
+// division, which a warp executes only if one of its lanes needs it.
+// The IEEE-division fallback of quotients_by_scale, out of line: it runs
+// only for groups or elements outside the fast path's range.
+struct Quot16 {
+  float v[16];
+};
+
+__device__ __noinline__ Quot16 quotients_ieee(uint4 v0, uint4 v1, float scale, bool group_fast, Quot16 q) {
+  float f[16];
+  unpack8(v0, f);
+  unpack8(v1, f + 8);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t mag = __float_as_uint(f[i]) & 0x7FFFFFFFu;
+    if (!(group_fast && (mag >= 0x0B000000u || mag == 0u))) q.v[i] = __fdiv_rn(f[i], scale);
+  }
+  return q;
+}
+
+__device__ __forceinline__ void quotients_by_scale_ieee(const uint4& v0, const uint4& v1, float scale,
+                                                        bool group_fast, float* q) {
+  Quot16 in;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) in.v[i] = q[i];
+  const Quot16 out = quotients_ieee(v0, v1, scale, group_fast, in);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) q[i] = out.v[i];
+}
+
+__device__ __forceinline__ void quotients_by_scale(const uint4& v0, const uint4& v1, float scale,
+                                                   float* q) {
+  float f[16];
+  unpack8(v0, f);
+  unpack8(v1, f + 8);
+  const float r = __frcp_rn(scale);
+  const bool group_fast = scale >= 1.17549435e-38f && r <= 3.40282347e+38f;
+  bool any_slow = false;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t b = __float_as_uint(f[i]);
+    const uint32_t mag = b & 0x7FFFFFFFu;
+    any_slow |= !(group_fast && (mag >= 0x0B000000u || mag == 0u));
+    const float ax = __uint_as_float(mag);
+    const float q0 = __fmul_rn(ax, r);
+    const float e = fmaf(-q0, scale, ax);
+    q[i] = __uint_as_float(__float_as_uint(fmaf(e, r, q0)) | (b & 0x80000000u));
+  }
+  if (__any_sync(0xffffffffu, any_slow)) quotients_by_scale_ieee(v0, v1, scale, group_fast, q);
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(kMoveThreads)
 dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__ recv_x,
@@ -56,23 +118,27 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
       my_w = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
     }
     if constexpr (FP8) {
-      float f[16];
-      unpack8(v0, f);
-      unpack8(v1, f + 8);
       float amax = 0.0f;
+      {
+        float f[16];
+        unpack8(v0, f);
+        unpack8(v1, f + 8);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      }
       // 8 consecutive lanes hold one 128-channel group
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
       float scale = __fdiv_rn(amax, kE4M3Max);
       if (scale == 0.0f) scale = 1.0f;
+      float f[16];
+      quotients_by_scale(v0, v1, scale, f);
       uint32_t q[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = pack_e4m3x2(__fdiv_rn(f[4 * i + 0], scale), __fdiv_rn(f[4 * i + 1], scale));
-        const uint32_t hi = pack_e4m3x2(__fdiv_rn(f[4 * i + 2], scale), __fdiv_rn(f[4 * i + 3], scale));
+        const uint32_t lo = pack_e4m3x2(f[4 * i + 0], f[4 * i + 1]);
+        const uint32_t hi = pack_e4m3x2(f[4 * i + 2], f[4 * i + 3]);
         q[i] = lo | (hi << 16);
       }
       const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
