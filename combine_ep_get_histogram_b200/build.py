@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libep_b200.so")
-SOURCES = ["ep_api.cu"]
+SOURCES = ["ep_api.cu", "ep_noalloc.cu"]
 DEPS = ["common.cuh", "layout.cuh", "movement.cuh"]
 
 NVCC_FLAGS = [

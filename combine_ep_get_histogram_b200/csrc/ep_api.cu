@@ -340,6 +340,9 @@ const char* ep_status_string(int status) {
     case EP_ERR_BAD_INDEX: return "EP_ERR_BAD_INDEX: a topk_idx entry outside [-1, E)";
     case EP_ERR_CUDA: return "EP_ERR_CUDA: a CUDA call or kernel launch failed";
     case EP_ERR_UNSUPPORTED: return "EP_ERR_UNSUPPORTED: the current device is not an sm_100 GPU";
+    case EP_ERR_SCRATCH_TOO_SMALL:
+      return "EP_ERR_SCRATCH_TOO_SMALL: the shape needs more layout scratch than the no-alloc entry point's "
+             "fixed array holds (ep_noalloc_scratch_bytes)";
     default: return "unknown ep status";
   }
 }

@@ -20,6 +20,7 @@ import os
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep_b200.so")
 
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_INDEX, EP_ERR_CUDA, EP_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
+EP_ERR_SCRATCH_TOO_SMALL = 5
 
 HANDLE_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank",
                  "count_src_rank_expert", "src_rank_expert_offset", "is_token_in_rank",
@@ -27,7 +28,8 @@ HANDLE_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank"
 
 EXPORTED = ("ep_handle_sizes", "ep_workspace_size", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_combine_backward", "ep_dispatch_backward", "ep_get_error",
-            "ep_status_string", "ep_last_cuda_error")
+            "ep_status_string", "ep_last_cuda_error", "ep_get_dispatch_layout_noalloc",
+            "ep_noalloc_scratch_bytes")
 
 
 class ep_shape_t(ctypes.Structure):
@@ -69,6 +71,8 @@ def _lib():
             "ep_get_error": (ctypes.c_int, [hp, vp]),
             "ep_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "ep_last_cuda_error": (ctypes.c_char_p, []),
+            "ep_get_dispatch_layout_noalloc": (ctypes.c_int, [shp, vp, hp, vp]),
+            "ep_noalloc_scratch_bytes": (ctypes.c_size_t, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -157,6 +161,15 @@ def ep_get_dispatch_layout(shape: ep_shape_t, topk_idx, handle: Handle, ws, stre
     st = _lib().ep_get_dispatch_layout(ctypes.byref(shape), _ptr(topk_idx), ctypes.byref(handle.c),
                                        _ptr(ws), nbytes, _stream(stream))
     return _check(st, "ep_get_dispatch_layout") if check else st
+
+
+def ep_get_dispatch_layout_noalloc(shape: ep_shape_t, topk_idx, handle: Handle, stream=None,
+                                   check=True) -> int:
+    """The layout with the library's fixed scratch array instead of a caller
+    workspace, for callers that cannot allocate device memory (see ep.h)."""
+    st = _lib().ep_get_dispatch_layout_noalloc(ctypes.byref(shape), _ptr(topk_idx), ctypes.byref(handle.c),
+                                               _stream(stream))
+    return _check(st, "ep_get_dispatch_layout_noalloc") if check else st
 
 
 def ep_dispatch(shape: ep_shape_t, x, topk_weights, handle: Handle, recv_x, recv_scale=None,

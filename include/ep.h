@@ -77,7 +77,9 @@ typedef enum {
   EP_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, shape outside the limits */
   EP_ERR_BAD_INDEX = 2,    /* a topk_idx entry outside [-1, E) (from ep_get_error) */
   EP_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
-  EP_ERR_UNSUPPORTED = 4   /* the current device is not an sm_100 GPU */
+  EP_ERR_UNSUPPORTED = 4,  /* the current device is not an sm_100 GPU */
+  EP_ERR_SCRATCH_TOO_SMALL = 5 /* the shape needs more layout scratch than
+                                  ep_get_dispatch_layout_noalloc's fixed array */
 } ep_status_t;
 
 /* Problem shape. T tokens over R virtual ranks, hidden H, top-k, E experts. */
@@ -140,6 +142,32 @@ int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const voi
 /* Backward of dispatch: grad_recv [P,H] bf16 -> grad_x [T,H] bf16. */
 int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv,
                          const ep_handle_t* handle, void* grad_x, ep_stream_t stream);
+
+/* ep_get_dispatch_layout without caller-provided scratch.  The pages describe
+ * no such call (it has no counterpart there); it exists for callers that
+ * cannot allocate device memory: code running while a CUDA graph is being
+ * captured, code inside another framework's allocator or memory-pool hooks,
+ * and hosts whose device memory is fixed at start-up.  The scratch comes from
+ * one fixed array of ep_noalloc_scratch_bytes() (1 MiB) inside the library,
+ * which every GPU that loads the library keeps until the process exits.
+ *  - Same arguments, results and errors as ep_get_dispatch_layout, minus the
+ *    workspace.  Returns EP_ERR_SCRATCH_TOO_SMALL, and enqueues nothing, when
+ *    ep_workspace_size(shape) exceeds the array (the limit is about 1000
+ *    layout tiles x (E + R) columns, e.g. T = 32768, E = 256, R = 8 needs
+ *    271 KiB).
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; nothing in it needs to start at zero.  Calls whose kernels
+ *    overlap on the GPU (other streams, other threads) race on it: order
+ *    them on one stream or serialise them. */
+int ep_get_dispatch_layout_noalloc(const ep_shape_t* shape, const int64_t* topk_idx,
+                                   const ep_handle_t* handle, ep_stream_t stream);
+
+/* Size in bytes of ep_get_dispatch_layout_noalloc's fixed scratch array. */
+size_t ep_noalloc_scratch_bytes(void);
 
 /* Synchronises `stream`, reads handle->error_word, clears it, and returns
  * EP_ERR_BAD_INDEX if a bad expert id was seen since the last call, EP_OK if
