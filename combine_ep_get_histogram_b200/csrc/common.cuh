@@ -19,6 +19,7 @@ constexpr int kTileFlagBytes = 32768;         // layout tile: tokens x ranks fla
 constexpr int kLayoutThreads = 256;
 constexpr int kLayoutWarps = kLayoutThreads / kWarp;
 constexpr int kMaxChunksPerWarp = (kTilePairs / kLayoutWarps + kWarp - 1) / kWarp;  // 4
+constexpr int kPairsPerThread = kTilePairs / kLayoutThreads;                         // 4
 constexpr float kE4M3Max = 448.0f;
 
 // 16-byte load of data that no thread writes during the kernel: non-coherent
@@ -32,8 +33,31 @@ __device__ __forceinline__ uint4 ld_ro_v4(const void* p) {
   return v;
 }
 
+// 16-byte load of read-only data that other warps of the CTA read too: cached in L1.
+__device__ __forceinline__ uint4 ld_l1_v4(const void* p) {
+  uint4 v;
+  asm("ld.global.ca.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
   *reinterpret_cast<uint4*>(p) = v;
+}
+
+// L2 policy that marks written lines first in line for eviction.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte store with an L2 cache policy.  No memory clobber: callers use it
+// only for outputs that no load of the same kernel reads.
+__device__ __forceinline__ void st_v4_hint(void* p, uint4 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;"
+               :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy));
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }

@@ -38,7 +38,9 @@ struct DeviceInfo {
   int sms = 0;
   bool supported = false;
   int occ_count = 0, occ_scan = 0, occ_assign = 0;
-  int occ_disp_bf16 = 0, occ_disp_fp8 = 0, occ_comb = 0, occ_dbwd = 0, occ_cbwd8 = 0, occ_cbwd32 = 0;
+  int occ_disp_bf16 = 0, occ_disp_fp8 = 0, occ_comb = 0, occ_dbwd = 0;
+  int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
+  int occ_cbwd = 0;
 };
 
 constexpr int kMaxDevices = 64;
@@ -66,15 +68,15 @@ int device_info(const DeviceInfo** out) {
     d.sms = prop.multiProcessorCount;
     d.supported = prop.major == 10 && prop.minor == 0;
     if (d.supported) {
+      cudaFuncSetAttribute(reinterpret_cast<const void*>(layout_small_kernel),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallMaxSmem);
       d.occ_count = occupancy(reinterpret_cast<const void*>(layout_count_kernel), kLayoutThreads,
                               (kMaxE + kMaxR) * 4 + kTileFlagBytes);
       d.occ_disp_bf16 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<false>), kMoveThreads, 0);
       d.occ_disp_fp8 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<true>), kMoveThreads, 0);
       d.occ_comb = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<true>), kMoveThreads, 0);
       d.occ_dbwd = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false>), kMoveThreads, 0);
-      d.occ_cbwd8 = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<8>), kMoveThreads, 0);
-      d.occ_cbwd32 =
-          occupancy(reinterpret_cast<const void*>(combine_backward_kernel<kMaxK>), kMoveThreads, 0);
+      d.occ_cbwd = occupancy(reinterpret_cast<const void*>(combine_backward_kernel), kMoveThreads, 0);
       cudaGetLastError();
     }
     g_dev[dev] = d;
@@ -222,6 +224,10 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
   p.error_word = handle->error_word;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
+    layout_small_kernel<<<1, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s>>>(p);
+    return finish(handle, s);
+  }
   if (g.nt > 0) {
     const size_t smem = static_cast<size_t>(g.ncol) * 4 + static_cast<size_t>(g.tile_t) * shape->R;
     layout_count_kernel<<<g.nt, kLayoutThreads, smem, s>>>(p);
@@ -247,7 +253,31 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
   const MoveParams p = move_params(shape, handle, topk_weights);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t units = T * p.chunks;
-  if (shape->use_fp8) {
+  if (p.chunks >= kTmaMinChunks && p.chunks <= kTmaMaxChunks) {
+    const bool fp8 = shape->use_fp8 != 0;
+    const int threads = p.chunks * kWarp;
+    const size_t smem = tma_smem_layout(shape->H, fp8).total;
+    const void* fn = fp8 ? reinterpret_cast<const void*>(dispatch_tma_kernel<true>)
+                         : reinterpret_cast<const void*>(dispatch_tma_kernel<false>);
+    int occ;
+    {
+      std::lock_guard<std::mutex> lock(g_dev_mu);
+      int& cached = const_cast<DeviceInfo*>(d)->occ_tma[fp8][p.chunks];
+      if (cached == 0) cached = occupancy(fn, threads, smem);
+      occ = cached;
+    }
+    // Large batches run 2 CTAs per SM (fewer row copies in flight per SM
+    // measured faster at 32768 tokens); small ones use every resident slot.
+    if (T >= 16 * static_cast<int64_t>(d->sms) && occ > 2) occ = 2;
+    const int64_t cap = grid_cap(*d, shape, occ);
+    const int grid = static_cast<int>(T < cap ? T : cap);
+    if (fp8)
+      dispatch_tma_kernel<true><<<grid, threads, smem, s>>>(p, static_cast<const uint16_t*>(x), recv_x, recv_scale,
+                                                             recv_weight);
+    else
+      dispatch_tma_kernel<false><<<grid, threads, smem, s>>>(p, static_cast<const uint16_t*>(x), recv_x, nullptr,
+                                                              recv_weight);
+  } else if (shape->use_fp8) {
     dispatch_kernel<true><<<movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s>>>(
         p, static_cast<const uint16_t*>(x), recv_x, recv_scale, recv_weight);
   } else {
@@ -289,17 +319,9 @@ int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const voi
   if (T == 0) return EP_OK;
   const MoveParams p = move_params(shape, handle, topk_weights);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const bool small_k = shape->k <= 8;
-  const int64_t cap = grid_cap(*d, shape, small_k ? d->occ_cbwd8 : d->occ_cbwd32);
-  const int grid = static_cast<int>(T < cap ? T : cap);
-  if (small_k)
-    combine_backward_kernel<8><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_out),
-                                                             static_cast<const uint16_t*>(y),
-                                                             static_cast<uint16_t*>(grad_y), grad_w);
-  else
-    combine_backward_kernel<kMaxK><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_out),
-                                                                 static_cast<const uint16_t*>(y),
-                                                                 static_cast<uint16_t*>(grad_y), grad_w);
+  combine_backward_kernel<<<movement_grid(*d, shape, d->occ_cbwd, T * shape->k), kMoveThreads, 0, s>>>(
+      p, static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y), static_cast<uint16_t*>(grad_y),
+      grad_w);
   return finish(handle, s);
 }
 

@@ -15,14 +15,16 @@
 //      (tokens with >= 1 pair there); writes is_token_in_rank rows and the
 //      tile's column of the [E+R, tiles] count matrix.
 //   2. layout_scan_kernel: one CTA per column: exclusive scan over tiles in
-//      place, column total on the side.
+//      place; the column's total and summaries (num_tokens_per_expert,
+//      num_tokens_per_rank, count_src_rank_expert, and the per-rank offsets
+//      relative to the expert's first row).
 //   3. layout_assign_kernel: one CTA per tile: exclusive scan of the expert
 //      totals (expert_offset), then the tile's pairs are ranked in (t, j)
 //      order: each warp owns a contiguous run of pairs, counts it per
 //      expert, the eight warp counts are scanned per expert from the tile's
 //      base, and each warp walks its run again giving lane l of a 32-pair
-//      chunk the rank popc(same_expert_mask & lanemask_lt).  CTA 0 also
-//      writes the per-rank and per-(rank, expert) summaries.
+//      chunk the rank popc(same_expert_mask & lanemask_lt).  The CTAs also
+//      add expert_offset to the per-(rank, expert) offsets, a slice each.
 #pragma once
 
 #include "common.cuh"
@@ -72,30 +74,39 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutPara
   tile_range(p, tile, t0, t1);
   const int ntok = t1 - t0;
   const int npairs = ntok * p.k;
-  for (int i = threadIdx.x; i < p.ncol; i += blockDim.x) hist[i] = 0;
-  for (int i = threadIdx.x; i < ntok * p.R; i += blockDim.x) flags[i] = 0;
-  __syncthreads();
-
   bool bad = false;
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t* idx = p.topk_idx + static_cast<int64_t>(t0) * p.k;
-  for (int base = 0; base < npairs; base += blockDim.x) {  // uniform trip count
-    const int i = base + threadIdx.x;
-    int e = -1;
-    if (i < npairs) e = pair_expert(p, idx[i], bad);
-    const unsigned same = __match_any_sync(0xffffffffu, e);
-    if (e >= 0) {
-      if (lane == __ffs(same) - 1) atomicAdd(&hist[e], __popc(same));
-      flags[(i / p.k) * p.R + e / p.Er] = 1;
+  // a tile holds at most kTilePairs pairs: every thread loads its (up to)
+  // kPairsPerThread expert ids first, then counts them
+  int e[kPairsPerThread];
+#pragma unroll
+  for (int c = 0; c < kPairsPerThread; ++c) {
+    const int i = c * kLayoutThreads + threadIdx.x;
+    e[c] = i < npairs ? pair_expert(p, idx[i], bad) : -1;
+  }
+  for (int i = threadIdx.x; i < p.ncol; i += blockDim.x) hist[i] = 0;
+  for (int i = threadIdx.x; i < ntok * p.R; i += blockDim.x) flags[i] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < kPairsPerThread; ++c) {
+    const int i = c * kLayoutThreads + threadIdx.x;
+    const unsigned same = __match_any_sync(0xffffffffu, e[c]);
+    if (e[c] >= 0) {
+      if (lane == __ffs(same) - 1) atomicAdd(&hist[e[c]], __popc(same));
+      flags[(i / p.k) * p.R + e[c] / p.Er] = 1;
     }
   }
   __syncthreads();
 
   uint8_t* itr = p.is_token_in_rank + static_cast<int64_t>(t0) * p.R;
-  for (int i = threadIdx.x; i < ntok * p.R; i += blockDim.x) {
-    const uint8_t f = flags[i];
-    itr[i] = f;
-    if (f) atomicAdd(&hist[p.E + i % p.R], 1);
+  for (int base = 0; base < ntok * p.R; base += blockDim.x) {  // uniform trip count
+    const int i = base + threadIdx.x;
+    const uint8_t f = i < ntok * p.R ? flags[i] : 0;
+    if (i < ntok * p.R) itr[i] = f;
+    const int key = f ? i % p.R : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[p.E + key], __popc(same));
   }
   __syncthreads();
   for (int c = threadIdx.x; c < p.ncol; c += blockDim.x)
@@ -148,6 +159,19 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scan_kernel(LayoutParam
   int32_t* col = p.colhist + static_cast<int64_t>(c) * p.nt;
   const int32_t total = block_exclusive_scan(col, p.nt, scratch);
   if (threadIdx.x == 0) p.coltotal[c] = total;
+  if (c < p.E) {
+    // expert column: totals, and per source rank the pairs before the rank's
+    // first tile (offsets relative to expert_offset[c]; the assign kernel adds it)
+    if (threadIdx.x == 0) p.num_tokens_per_expert[c] = total;
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+      const int32_t pre = p.tiles_per_rank > 0 ? col[r * p.tiles_per_rank] : 0;
+      const int32_t nxt = (r + 1 < p.R && p.tiles_per_rank > 0) ? col[(r + 1) * p.tiles_per_rank] : total;
+      p.src_rank_expert_offset[r * p.E + c] = pre;
+      p.count_src_rank_expert[r * p.E + c] = nxt - pre;
+    }
+  } else if (threadIdx.x == 0) {
+    p.num_tokens_per_rank[c - p.E] = total;
+  }
 }
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutParams p) {
@@ -156,69 +180,70 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
   int32_t* whist = smem + p.E + 1;            // [kLayoutWarps * E]
   __shared__ int32_t scratch[kWarp];
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
+  const int tile = blockIdx.x;
+  const bool has_tile = tile < p.nt;
+
+  // issue the tile's loads first: its pairs' expert ids (each warp owns the
+  // contiguous run [w*S, min((w+1)*S, npairs)), S a multiple of 32) and its
+  // per-expert base within each expert block
+  int t0 = 0, t1 = 0;
+  if (has_tile) tile_range(p, tile, t0, t1);
+  const int npairs = (t1 - t0) * p.k;
+  const int64_t pair0 = static_cast<int64_t>(t0) * p.k;
+  const int S = ((npairs + kLayoutWarps - 1) / kLayoutWarps + kWarp - 1) / kWarp * kWarp;
+  const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
+  int ereg[kMaxChunksPerWarp];
+  bool bad = false;  // already reported by layout_count_kernel
+#pragma unroll
+  for (int c = 0; c < kMaxChunksPerWarp; ++c) {
+    const int i = my_lo + c * kWarp + lane;
+    ereg[c] = i < my_hi ? pair_expert(p, p.topk_idx[pair0 + i], bad) : -1;
+  }
+  int32_t tile_base[kMaxE / kLayoutThreads];
+#pragma unroll
+  for (int c = 0; c < kMaxE / kLayoutThreads; ++c) {
+    const int e = c * kLayoutThreads + threadIdx.x;
+    tile_base[c] = (has_tile && e < p.E) ? p.colhist[static_cast<int64_t>(e) * p.nt + tile] : 0;
+  }
 
   // expert_offset = exclusive scan of the expert totals (every CTA)
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) eoff[e] = p.coltotal[e];
+  for (int i = threadIdx.x; i < kLayoutWarps * p.E; i += blockDim.x) whist[i] = 0;
   __syncthreads();
   const int32_t p_eff = block_exclusive_scan(eoff, p.E, scratch);
   if (threadIdx.x == 0) eoff[p.E] = p_eff;
   __syncthreads();
 
-  if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
-      p.expert_offset[e] = eoff[e];
-      if (e < p.E) p.num_tokens_per_expert[e] = p.coltotal[e];
-    }
-    for (int r = threadIdx.x; r < p.R; r += blockDim.x) p.num_tokens_per_rank[r] = p.coltotal[p.E + r];
-    for (int i = threadIdx.x; i < p.R * p.E; i += blockDim.x) {
-      const int r = i / p.E, e = i - r * p.E;
-      const int32_t* col = p.colhist + static_cast<int64_t>(e) * p.nt;
-      const int32_t pre = p.tiles_per_rank > 0 ? col[r * p.tiles_per_rank] : 0;
-      const int32_t nxt = (r + 1 < p.R && p.tiles_per_rank > 0) ? col[(r + 1) * p.tiles_per_rank]
-                                                                : p.coltotal[e];
-      p.src_rank_expert_offset[i] = eoff[e] + pre;
-      p.count_src_rank_expert[i] = nxt - pre;
-    }
-  }
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.expert_offset[e] = eoff[e];
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.R * p.E; i += gridDim.x * blockDim.x)
+    p.src_rank_expert_offset[i] += eoff[i % p.E];
   // rows past the last valid pair have no source
   const int64_t P = static_cast<int64_t>(p.T) * p.k;
   for (int64_t i = p_eff + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < P;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     p.src_of_slot[i] = -1;
+  if (!has_tile) return;
 
-  const int tile = blockIdx.x;
-  if (tile >= p.nt) return;
-  int t0, t1;
-  tile_range(p, tile, t0, t1);
-  const int npairs = (t1 - t0) * p.k;
-  const int64_t pair0 = static_cast<int64_t>(t0) * p.k;
-
-  for (int i = threadIdx.x; i < kLayoutWarps * p.E; i += blockDim.x) whist[i] = 0;
-  __syncthreads();
-
-  // each warp owns pairs [w*S, min((w+1)*S, npairs)), S a multiple of 32
-  const int S = ((npairs + kLayoutWarps - 1) / kLayoutWarps + kWarp - 1) / kWarp * kWarp;
-  const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
   int32_t* wh = whist + warp * p.E;
-  int ereg[kMaxChunksPerWarp];
-  bool bad = false;
 #pragma unroll
   for (int c = 0; c < kMaxChunksPerWarp; ++c) {
-    const int i = my_lo + c * kWarp + lane;
-    int e = -1;
-    if (i < my_hi) e = pair_expert(p, p.topk_idx[pair0 + i], bad);
-    ereg[c] = e;
+    const int e = ereg[c];
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
     __syncwarp();
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
-    int32_t run = eoff[e] + p.colhist[static_cast<int64_t>(e) * p.nt + tile];
-    for (int w = 0; w < kLayoutWarps; ++w) {
-      const int32_t c = whist[w * p.E + e];
-      whist[w * p.E + e] = run;
-      run += c;
+#pragma unroll
+  for (int c = 0; c < kMaxE / kLayoutThreads; ++c) {
+    const int e = c * kLayoutThreads + threadIdx.x;
+    if (e < p.E) {
+      int32_t run = eoff[e] + tile_base[c];
+      for (int w = 0; w < kLayoutWarps; ++w) {
+        const int32_t n = whist[w * p.E + e];
+        whist[w * p.E + e] = run;
+        run += n;
+      }
     }
   }
   __syncthreads();
@@ -239,6 +264,140 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
     if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
     __syncwarp();
   }
+}
+
+// ------------------------------------------------- small problems, one CTA
+//
+// For up to kSmallMaxPairs pairs the whole layout fits one CTA of 32 warps,
+// and one launch replaces the three above (the decode shape, 8 ranks x 128
+// tokens x top-8, is 8192 pairs).  The same counting sort with the CTA as the
+// only tile: each warp owns a contiguous run of pairs; per-warp expert
+// histograms are scanned per expert in warp order from the expert's first
+// row; pairs are ranked with popc(same_expert_mask & lanemask_lt).
+// Per-(source rank, expert) counts and per-rank token counts are warp-
+// aggregated shared-memory atomics (their sums do not depend on order);
+// is_token_in_rank is a shared-memory flag array written out at the end.
+
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / kWarp;
+constexpr int kSmallMaxPairs = 16384;
+constexpr int kSmallMaxE = 256;
+constexpr int kSmallMaxR = 64;
+constexpr int kSmallMaxRE = 2048;
+constexpr int kSmallMaxFlags = 16384;  // T x R token-rank flags (bytes)
+constexpr int kSmallChunks = kSmallMaxPairs / kSmallThreads;  // 32-pair chunks per warp
+constexpr int kSmallMaxSmem = (kSmallWarps * kSmallMaxE + kSmallMaxE + 1 + kSmallMaxRE + kSmallMaxR) * 4 +
+                              kSmallMaxFlags;
+
+__host__ __device__ inline bool layout_small_fits(int T, int k, int E, int R) {
+  return static_cast<int64_t>(T) * k <= kSmallMaxPairs && E <= kSmallMaxE && R <= kSmallMaxR &&
+         R * E <= kSmallMaxRE && static_cast<int64_t>(T) * R <= kSmallMaxFlags;
+}
+
+__host__ __device__ inline int layout_small_smem(int T, int E, int R) {
+  return (kSmallWarps * E + (E + 1) + R * E + R) * 4 + T * R;
+}
+
+__global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutParams p) {
+  extern __shared__ int32_t smem[];
+  int32_t* whist = smem;                          // [32][E]
+  int32_t* eoff = whist + kSmallWarps * p.E;      // [E + 1]
+  int32_t* cnt = eoff + p.E + 1;                  // [R][E] pairs by (source rank, expert)
+  int32_t* rank_cnt = cnt + p.R * p.E;            // [R]
+  uint8_t* flags = reinterpret_cast<uint8_t*>(rank_cnt + p.R);  // [T][R]
+  __shared__ int32_t scratch[kWarp];
+  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
+  const int P = p.T * p.k;
+  const int S = ((P + kSmallWarps - 1) / kSmallWarps + kWarp - 1) / kWarp * kWarp;
+  const int my_lo = warp * S, my_hi = min(my_lo + S, P);
+
+  bool bad = false;
+  int ereg[kSmallChunks];
+#pragma unroll
+  for (int c = 0; c < kSmallChunks; ++c) {
+    const int i = my_lo + c * kWarp + lane;
+    ereg[c] = i < my_hi ? pair_expert(p, p.topk_idx[i], bad) : -1;
+  }
+  for (int i = threadIdx.x; i < kSmallWarps * p.E; i += blockDim.x) whist[i] = 0;
+  for (int i = threadIdx.x; i < p.R * p.E + p.R; i += blockDim.x) cnt[i] = 0;  // cnt and rank_cnt
+  for (int i = threadIdx.x; i < p.T * p.R; i += blockDim.x) flags[i] = 0;
+  __syncthreads();
+
+  int32_t* wh = whist + warp * p.E;
+#pragma unroll
+  for (int c = 0; c < kSmallChunks; ++c) {
+    const int i = my_lo + c * kWarp + lane;
+    const int e = ereg[c];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
+    const int key = e >= 0 ? (i / p.k / p.Tr) * p.E + e : -1;
+    const unsigned same_key = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(same_key) - 1) atomicAdd(&cnt[key], __popc(same_key));
+    if (e >= 0) flags[(i / p.k) * p.R + e / p.Er] = 1;
+    __syncwarp();
+  }
+  __syncthreads();
+
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+    int32_t tot = 0;
+    for (int w = 0; w < kSmallWarps; ++w) tot += whist[w * p.E + e];
+    eoff[e] = tot;
+    p.num_tokens_per_expert[e] = tot;
+  }
+  __syncthreads();
+  const int32_t p_eff = block_exclusive_scan(eoff, p.E, scratch);
+  if (threadIdx.x == 0) eoff[p.E] = p_eff;
+  __syncthreads();
+  for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
+    p.expert_offset[e] = eoff[e];
+    if (e == p.E) break;
+    int32_t run = eoff[e];
+    for (int w = 0; w < kSmallWarps; ++w) {
+      const int32_t n = whist[w * p.E + e];
+      whist[w * p.E + e] = run;
+      run += n;
+    }
+    run = eoff[e];
+    for (int r = 0; r < p.R; ++r) {
+      const int32_t n = cnt[r * p.E + e];
+      p.src_rank_expert_offset[r * p.E + e] = run;
+      p.count_src_rank_expert[r * p.E + e] = n;
+      run += n;
+    }
+  }
+  __syncthreads();
+
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int c = 0; c < kSmallChunks; ++c) {
+    const int i = my_lo + c * kWarp + lane;
+    const int e = ereg[c];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int32_t s = wh[e] + __popc(same & lt);
+      p.slot_of_pair[i] = s;
+      p.src_of_slot[s] = i;
+    } else if (i < my_hi) {
+      p.slot_of_pair[i] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
+    __syncwarp();
+  }
+  for (int i = p_eff + threadIdx.x; i < P; i += blockDim.x) p.src_of_slot[i] = -1;
+
+  // is_token_in_rank and per-rank token counts from the flags
+  for (int base = 0; base < p.T * p.R; base += blockDim.x) {  // uniform trip count
+    const int i = base + threadIdx.x;
+    const uint8_t f = i < p.T * p.R ? flags[i] : 0;
+    if (i < p.T * p.R) p.is_token_in_rank[i] = f;
+    const int key = f ? i % p.R : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&rank_cnt[key], __popc(same));
+  }
+  __syncthreads();
+  for (int r = threadIdx.x; r < p.R; r += blockDim.x) p.num_tokens_per_rank[r] = rank_cnt[r];
+  if (bad) atomicOr(p.error_word, 1);
 }
 
 }  // namespace ep

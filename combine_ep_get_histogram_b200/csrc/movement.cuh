@@ -33,19 +33,6 @@ constexpr int kMoveWarps = kMoveThreads / kWarp;
 
 // ---------------------------------------------------------------- dispatch
 
-// f[i] <- x_i / scale, rounded to nearest even in fp32, for 16 values of one
-// 128-channel group (scale >= the group's amax / 448).
-//
-// Fast path (Markstein's division with a correctly rounded reciprocal, P.
-// Markstein, "Computation of elementary functions on the IBM RISC System/6000
-// processor", IBM J. Res. Dev. 34(1), 1990): r = RN(1/scale), q0 = RN(|x|*r),
-// e = |x| - q0*scale (exact through the FMA), q = RN(q0 + e*r), sign copied
-// back.  It gives the correctly rounded quotient unless the remainder
-// underflows; for inputs that are bf16 values this holds whenever |x| >=
-// 2^-105 and scale is a normal number with a finite reciprocal.  Every
-// (x, amax) pair of bf16 values was checked: the resulting E4M3 codes equal
-// those of the IEEE division.  Other elements (zeros excepted) take the IEEE
-// division, which a warp executes only if one of its lanes needs it.
 // The IEEE-division fallback of quotients_by_scale, out of line: it runs
 // only for groups or elements outside the fast path's range.
 struct Quot16 {
@@ -74,6 +61,19 @@ __device__ __forceinline__ void quotients_by_scale_ieee(const uint4& v0, const u
   for (int i = 0; i < 16; ++i) q[i] = out.v[i];
 }
 
+// q[i] <- x_i / scale, rounded to nearest even in fp32, for the 16 values of one
+// 128-channel group (scale >= the group's amax / 448).
+//
+// Fast path (Markstein's division with a correctly rounded reciprocal, P.
+// Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): r = RN(1/scale), q0 = RN(|x|*r),
+// e = |x| - q0*scale (exact through the FMA), q = RN(q0 + e*r), sign copied
+// back.  It gives the correctly rounded quotient unless the remainder
+// underflows; for inputs that are bf16 values this holds whenever |x| >=
+// 2^-105 and scale is a normal number with a finite reciprocal.  Every
+// (x, amax) pair of bf16 values was checked: the resulting E4M3 codes equal
+// those of the IEEE division.  Other elements (zeros excepted) take the IEEE
+// division, which a warp executes only if one of its lanes needs it.
 __device__ __forceinline__ void quotients_by_scale(const uint4& v0, const uint4& v1, float scale,
                                                    float* q) {
   float f[16];
@@ -166,6 +166,146 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
   }
 }
 
+// ------------------------------------------------- dispatch, TMA row stores
+//
+// One CTA per token (grid-stride over tokens), one warp per 512-channel chunk
+// (4 <= chunks <= 16, i.e. 1536 < H <= 8192).  Each token's payload row (E4M3
+// codes, or the bf16 row itself) is assembled in shared memory and written to
+// its k receive rows by k TMA bulk copies (cp.async.bulk global <- shared)
+// issued by one thread, so every destination row is written as one
+// contiguous H- or 2H-byte transfer instead of 512-byte pieces from many
+// warps.  Two row stages alternate; before a stage is rewritten, the issuing
+// thread waits until the bulk copies of two tokens ago have finished reading
+// it (cp.async.bulk.wait_group.read).  The next token's x is loaded into
+// registers while the current one is quantised and stored.  Scales and gate
+// weights are written with plain stores from shared memory.
+
+constexpr int kTmaMinChunks = 4;
+constexpr int kTmaMaxChunks = 16;
+
+struct TmaSmemLayout {
+  int row_bytes;   // payload row bytes, rounded up to 128
+  int off_slot;    // int32 [2][kMaxK]
+  int off_w;       // float [2][kMaxK]
+  int off_scale;   // float [2][G]
+  int total;
+};
+
+__host__ __device__ inline TmaSmemLayout tma_smem_layout(int H, bool fp8) {
+  TmaSmemLayout L;
+  const int row = fp8 ? H : 2 * H;
+  L.row_bytes = (row + 127) / 128 * 128;
+  L.off_slot = 2 * L.row_bytes;
+  L.off_w = L.off_slot + 2 * kMaxK * 4;
+  L.off_scale = L.off_w + 2 * kMaxK * 4;
+  L.total = L.off_scale + (fp8 ? 2 * (H / kGroup) * 4 : 0);
+  return L;
+}
+
+__device__ __forceinline__ void bulk_store_row(void* gdst, uint32_t ssrc, int bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               :: "l"(gdst), "r"(ssrc), "r"(bytes) : "memory");
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kTmaMaxChunks * kWarp, 3)
+dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__ recv_x,
+                    float* __restrict__ recv_scale, float* __restrict__ recv_weight) {
+  extern __shared__ __align__(128) uint8_t tma_smem[];
+  const TmaSmemLayout L = tma_smem_layout(p.H, FP8);
+  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
+  const int h0 = warp * kChunk + lane * kLaneElems;  // one chunk per warp
+  const bool a0 = h0 < p.H, a1 = h0 + 8 < p.H;
+  const int row_bytes = FP8 ? p.H : 2 * p.H;
+
+  uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+  int t = blockIdx.x;
+  if (t < p.T) {
+    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H + h0;
+    if (a0) v0 = ld_ro_v4(xr);
+    if (a1) v1 = ld_ro_v4(xr + 8);
+  }
+  for (int it = 0; t < p.T; ++it, t += gridDim.x) {
+    const int stage = it & 1;
+    uint8_t* row = tma_smem + stage * L.row_bytes;
+    int32_t* sslot = reinterpret_cast<int32_t*>(tma_smem + L.off_slot) + stage * kMaxK;
+    float* sw = reinterpret_cast<float*>(tma_smem + L.off_w) + stage * kMaxK;
+    float* sscale = reinterpret_cast<float*>(tma_smem + L.off_scale) + stage * p.G;
+
+    // prefetch the next token of this CTA
+    const int tn = t + gridDim.x;
+    uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+    if (tn < p.T) {
+      const uint16_t* xr = x + static_cast<int64_t>(tn) * p.H + h0;
+      if (a0) n0 = ld_ro_v4(xr);
+      if (a1) n1 = ld_ro_v4(xr + 8);
+    }
+    // the row stage is free once the copies issued two tokens ago have read it
+    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    if (warp == 0 && lane < p.k) {
+      sslot[lane] = p.slot_of_pair[static_cast<int64_t>(t) * p.k + lane];
+      sw[lane] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
+    }
+    __syncthreads();
+
+    if constexpr (FP8) {
+      float amax = 0.0f;
+      {
+        float f[16];
+        unpack8(v0, f);
+        unpack8(v1, f + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+      float scale = __fdiv_rn(amax, kE4M3Max);
+      if (scale == 0.0f) scale = 1.0f;
+      float f[16];
+      quotients_by_scale(v0, v1, scale, f);
+      uint32_t q[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        q[i] = pack_e4m3x2(f[4 * i + 0], f[4 * i + 1]) | (pack_e4m3x2(f[4 * i + 2], f[4 * i + 3]) << 16);
+      if (a0) {
+        *reinterpret_cast<uint4*>(row + h0) = make_uint4(q[0], q[1], q[2], q[3]);
+        if ((lane & (kLanesPerGroup - 1)) == 0) sscale[h0 / kGroup] = scale;
+      }
+    } else {
+      if (a0) *reinterpret_cast<uint4*>(row + 2 * h0) = v0;
+      if (a1) *reinterpret_cast<uint4*>(row + 2 * h0 + 16) = v1;
+    }
+    // make the generic-proxy shared-memory writes visible to the bulk copies
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+
+    if (threadIdx.x == 0) {
+      const uint32_t src = static_cast<uint32_t>(__cvta_generic_to_shared(row));
+      for (int j = 0; j < p.k; ++j) {
+        const int s = sslot[j];
+        if (s >= 0) bulk_store_row(static_cast<uint8_t*>(recv_x) + static_cast<int64_t>(s) * row_bytes, src,
+                                   row_bytes);
+      }
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    if constexpr (FP8) {
+      for (int i = threadIdx.x; i < p.k * p.G; i += blockDim.x) {
+        const int j = i / p.G, g = i - j * p.G;
+        const int s = sslot[j];
+        if (s >= 0) recv_scale[static_cast<int64_t>(s) * p.G + g] = sscale[g];
+      }
+    }
+    if (recv_weight != nullptr && threadIdx.x < p.k) {
+      const int s = sslot[threadIdx.x];
+      if (s >= 0) recv_weight[s] = sw[threadIdx.x];
+    }
+    v0 = n0;
+    v1 = n1;
+  }
+  if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // -------------------------------------------- combine / dispatch backward
 //
 // out[t] = bf16( chain over j of (WEIGHTED ? fmaf(w[t,j], y[slot], acc) : acc + y[slot]) )
@@ -235,99 +375,78 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
 
 // -------------------------------------------------------- combine backward
 //
-// One CTA per token (grid-stride).  Warps stride over the token's 512-channel
-// chunks; for every pair j each lane writes grad_y = bf16(w_j * g) for its 16
-// channels and accumulates the partial dot product g . y_j in fp32.  Partial
-// sums are reduced across lanes (xor shuffles) and then across warps in warp
-// order, so the result does not depend on scheduling.
+// One warp per (token t, top-k position j) pair, grid-stride over the pairs:
+// the warp streams the whole y[slot] row in and the whole grad_y[slot] row
+// out, kUnroll 512-channel chunks at a time, and reads g[t] through L1 (the
+// k warps of one token usually share a CTA, so g comes from DRAM once).
+// grad_y = bf16(w * g) (one fp32 product); the dot product g . y[slot]
+// accumulates in fp32 in channel order per lane, then across lanes with xor
+// shuffles, so grad_w needs no cross-warp reduction and does not depend on
+// scheduling.  grad_y is written with an L2 evict-first policy: it is not read
+// again here, and letting it leave L2 first keeps the y rows being read from
+// being pushed out.
 
-template <int KMAX>  // 8 (k <= 8) or kMaxK
+constexpr int kCbwdUnroll = 4;
+
 __global__ void __launch_bounds__(kMoveThreads)
 combine_backward_kernel(MoveParams p, const uint16_t* __restrict__ g, const uint16_t* __restrict__ y,
                         uint16_t* __restrict__ grad_y, float* __restrict__ grad_w) {
-  __shared__ float part[kMoveWarps][KMAX];
-  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
-  for (int t = blockIdx.x; t < p.T; t += gridDim.x) {
-    int my_slot = -1;
-    float my_w = 0.0f;
-    if (lane < p.k) {
-      my_slot = p.slot_of_pair[static_cast<int64_t>(t) * p.k + lane];
-      my_w = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
+  const uint64_t evict_first = l2_evict_first_policy();
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int64_t npairs = static_cast<int64_t>(p.T) * p.k;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < npairs;
+       u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
+    const int s = p.slot_of_pair[u];
+    if (s < 0) {  // masked pair: no row, zero weight gradient
+      if (lane == 0) grad_w[u] = 0.0f;
+      continue;
     }
-    float dot[KMAX];
+    const float w = p.topk_weights[u];
+    const int t = static_cast<int>(u / p.k);
+    const uint16_t* gr = g + static_cast<int64_t>(t) * p.H;
+    const uint16_t* yr = y + static_cast<int64_t>(s) * p.H;
+    uint16_t* dr = grad_y + static_cast<int64_t>(s) * p.H;
+    float d = 0.0f;
+    for (int c0 = 0; c0 < p.chunks; c0 += kCbwdUnroll) {
+      uint4 gv[kCbwdUnroll][2], yv[kCbwdUnroll][2];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) dot[j] = 0.0f;
-    for (int c = warp; c < p.chunks; c += kMoveWarps) {
-      const int h0 = c * kChunk + lane * kLaneElems;
-      const bool a0 = h0 < p.H, a1 = h0 + 8 < p.H;
-      const uint16_t* gr = g + static_cast<int64_t>(t) * p.H + h0;
-      uint4 gv0 = make_uint4(0, 0, 0, 0), gv1 = gv0;
-      if (a0) gv0 = ld_ro_v4(gr);
-      if (a1) gv1 = ld_ro_v4(gr + 8);
-      float gf[16];
-      unpack8(gv0, gf);
-      unpack8(gv1, gf + 8);
-#pragma unroll
-      for (int jb = 0; jb < KMAX; jb += 8) {
-        if (jb < p.k) {
-          uint4 v[8][2];
-          int s[8];
-          float w[8];
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            s[jj] = __shfl_sync(0xffffffffu, my_slot, jb + jj);
-            w[jj] = __shfl_sync(0xffffffffu, my_w, jb + jj);
-            if (jb + jj >= p.k) s[jj] = -1;
-          }
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            v[jj][0] = make_uint4(0, 0, 0, 0);
-            v[jj][1] = v[jj][0];
-            if (s[jj] >= 0) {
-              const uint16_t* src = y + static_cast<int64_t>(s[jj]) * p.H + h0;
-              if (a0) v[jj][0] = ld_ro_v4(src);
-              if (a1) v[jj][1] = ld_ro_v4(src + 8);
-            }
-          }
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            if (s[jj] >= 0) {
-              float yf[16], gy[16];
-              unpack8(v[jj][0], yf);
-              unpack8(v[jj][1], yf + 8);
-              float d = dot[jb + jj];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                gy[i] = __fmul_rn(w[jj], gf[i]);
-                d = fmaf(gf[i], yf[i], d);
-              }
-              dot[jb + jj] = d;
-              uint16_t* dst = grad_y + static_cast<int64_t>(s[jj]) * p.H + h0;
-              if (a0) st_v4(dst, pack8_bf16(gy));
-              if (a1) st_v4(dst + 8, pack8_bf16(gy + 8));
-            }
-          }
+      for (int q = 0; q < kCbwdUnroll; ++q) {
+        const int h0 = (c0 + q) * kChunk + lane * kLaneElems;
+        gv[q][0] = gv[q][1] = yv[q][0] = yv[q][1] = make_uint4(0, 0, 0, 0);
+        if (h0 < p.H) {
+          gv[q][0] = ld_l1_v4(gr + h0);
+          yv[q][0] = ld_ro_v4(yr + h0);
+        }
+        if (h0 + 8 < p.H) {
+          gv[q][1] = ld_l1_v4(gr + h0 + 8);
+          yv[q][1] = ld_ro_v4(yr + h0 + 8);
         }
       }
-    }
-    // reduce the partial dot products: lanes, then warps in order
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      if (j < p.k) {
-        float d = dot[j];
+      for (int q = 0; q < kCbwdUnroll; ++q) {
+        const int h0 = (c0 + q) * kChunk + lane * kLaneElems;
+        uint4 out[2];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-        if (lane == 0) part[warp][j] = d;
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t gw[4] = {gv[q][h].x, gv[q][h].y, gv[q][h].z, gv[q][h].w};
+          const uint32_t yw[4] = {yv[q][h].x, yv[q][h].y, yv[q][h].z, yv[q][h].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
+            d = fmaf(g0, bf16_lo(yw[i]), d);
+            d = fmaf(g1, bf16_hi(yw[i]), d);
+            o[i] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
+          }
+          out[h] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        if (h0 < p.H) st_v4_hint(dr + h0, out[0], evict_first);
+        if (h0 + 8 < p.H) st_v4_hint(dr + h0 + 8, out[1], evict_first);
       }
     }
-    __syncthreads();
-    if (threadIdx.x < p.k) {
-      const int j = threadIdx.x;
-      float d = 0.0f;
-      for (int w = 0; w < kMoveWarps; ++w) d += part[w][j];
-      grad_w[static_cast<int64_t>(t) * p.k + j] = my_slot >= 0 ? d : 0.0f;
-    }
-    __syncthreads();
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    if (lane == 0) grad_w[u] = d;
   }
 }
 

@@ -27,7 +27,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # EP_ORACLE_LIB names another build of ep_oracle.c; the mutation tests
+        # use it to check that the pins reject a deliberately wrong oracle.
+        path = os.environ.get("EP_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         i64, p = ctypes.c_int64, ctypes.c_void_p
         L.epo_e4m3_value.restype = ctypes.c_double

@@ -65,21 +65,25 @@ def random_idx(T, k, E, seed=0, masked=0.0, distinct=True):
     return np.ascontiguousarray(idx.astype(np.int64))
 
 
+# T*k <= 16384 (with E <= 256, R <= 64) takes the one-CTA layout kernel, larger
+# problems the three-kernel tiled one: the cases below run both.
+@pytest.mark.parametrize("T", [96, 4096])
 @pytest.mark.parametrize("use_fp8", [False, True])
-def test_masked_and_duplicate_pairs(cuda_device, use_fp8):
-    T, k, E, R = 96, 6, 24, 4
+def test_masked_and_duplicate_pairs(cuda_device, use_fp8, T):
+    k, E, R = 6, 24, 4
     idx = random_idx(T, k, E, seed=1, masked=0.25, distinct=False)
     idx[5] = -1  # a token with no pair
     idx[7] = 3   # one expert k times
     run_and_compare(cuda_device, T, 256, k, E, R, use_fp8, idx)
 
 
-def test_bad_index_flagged_and_masked(cuda_device):
-    T, k, E, R = 32, 4, 16, 2
+@pytest.mark.parametrize("T", [32, 8192])
+def test_bad_index_flagged_and_masked(cuda_device, T):
+    k, E, R = 4, 16, 2
     idx = random_idx(T, k, E, seed=2)
     idx[3, 1] = E
     idx[9, 0] = -7
-    idx[31, 3] = 1 << 40
+    idx[T - 1, 3] = 1 << 40
     path, ref = run_and_compare(cuda_device, T, 128, k, E, R, False, idx)
     assert oracle.layout(idx, E, R)["status"] == oracle.BAD_INDEX
     assert ep.ep_get_error(path.handle) == ep.ep.EP_ERR_BAD_INDEX
@@ -113,6 +117,10 @@ def test_empty_input(cuda_device):
     (64, 7176, 8, 32, 4, False),       # wide H with a ragged last chunk
     (32, 640, 8, 32, 4, True),         # FP8: one full chunk + one group
     (2400, 384, 8, 64, 8, True),       # 300 tokens per rank: ragged layout tiles
+    (2048, 2048, 8, 256, 8, False),    # largest one-CTA layout (16384 pairs), TMA BF16 dispatch
+    (2056, 2048, 8, 256, 8, True),     # just past it: tiled layout
+    (512, 8192, 8, 64, 8, True),       # widest TMA dispatch (16 warps)
+    (256, 8704, 4, 64, 8, False),      # past the TMA width: warp dispatch
 ])
 def test_shapes(cuda_device, T, H, k, E, R, use_fp8):
     run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=T + k))
