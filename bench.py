@@ -182,7 +182,8 @@ class Path:
 def launches_per_step(w) -> int:
     """Kernels one step launches: layout (one kernel for small problems, else
     count + scan + assign), dispatch, combine and the two backward passes."""
-    small = w.T * w.k <= 16384 and w.E <= 256 and w.R <= 64 and w.R * w.E <= 2048 and w.T * w.R <= 16384
+    small = (w.T * w.k <= 16384 and w.E <= 256 and w.R <= 64 and w.R * w.E <= 2048
+             and -(-w.T // 8) * w.R <= 8192)
     return (1 if small else 3) + 4
 
 

@@ -68,8 +68,6 @@ int device_info(const DeviceInfo** out) {
     d.sms = prop.multiProcessorCount;
     d.supported = prop.major == 10 && prop.minor == 0;
     if (d.supported) {
-      cudaFuncSetAttribute(reinterpret_cast<const void*>(layout_small_kernel),
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallMaxSmem);
       d.occ_count = occupancy(reinterpret_cast<const void*>(layout_count_kernel), kLayoutThreads,
                               (kMaxE + kMaxR) * 4 + kTileFlagBytes);
       d.occ_disp_bf16 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<false>), kMoveThreads, 0);
@@ -225,7 +223,7 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
-    layout_small_kernel<<<1, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s>>>(p);
+    layout_small_kernel<<<kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s>>>(p);
     return finish(handle, s);
   }
   if (g.nt > 0) {

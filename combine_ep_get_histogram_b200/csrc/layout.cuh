@@ -27,6 +27,8 @@
 //      add expert_offset to the per-(rank, expert) offsets, a slice each.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace ep {
@@ -266,138 +268,196 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
   }
 }
 
-// ------------------------------------------------- small problems, one CTA
+// ----------------------------------------- small problems, one CTA cluster
 //
-// For up to kSmallMaxPairs pairs the whole layout fits one CTA of 32 warps,
-// and one launch replaces the three above (the decode shape, 8 ranks x 128
-// tokens x top-8, is 8192 pairs).  The same counting sort with the CTA as the
-// only tile: each warp owns a contiguous run of pairs; per-warp expert
-// histograms are scanned per expert in warp order from the expert's first
-// row; pairs are ranked with popc(same_expert_mask & lanemask_lt).
-// Per-(source rank, expert) counts and per-rank token counts are warp-
-// aggregated shared-memory atomics (their sums do not depend on order);
-// is_token_in_rank is a shared-memory flag array written out at the end.
+// Up to kSmallMaxPairs pairs (the decode shape, 8 ranks x 128 tokens x
+// top-8, is 8192) are handled by one cluster of kClusterCtas CTAs on as many
+// SMs, in one launch.  CTA c takes the tile of whole tokens
+// [c*T/C, (c+1)*T/C).  Phase 1, per CTA: per-warp expert histograms of the
+// tile's pairs (each warp owns a contiguous run of pairs), per-(source rank,
+// expert) counts and per-rank token counts (warp-aggregated shared-memory
+// atomics, whose sums do not depend on order), is_token_in_rank.  Cluster
+// barrier.  Phase 2: every CTA reads the other tiles' histograms through
+// distributed shared memory, so it knows the expert totals (expert_offset)
+// and how many pairs of each expert come from earlier tiles; it scans its
+// warp histograms from there and ranks its pairs with
+// popc(same_expert_mask & lanemask_lt).  CTA 0 writes the summaries.  A
+// final cluster barrier keeps every CTA's shared memory alive until the
+// others have read it.
 
-constexpr int kSmallThreads = 1024;
+constexpr int kClusterCtas = 8;
+constexpr int kSmallThreads = 512;
 constexpr int kSmallWarps = kSmallThreads / kWarp;
 constexpr int kSmallMaxPairs = 16384;
 constexpr int kSmallMaxE = 256;
 constexpr int kSmallMaxR = 64;
 constexpr int kSmallMaxRE = 2048;
-constexpr int kSmallMaxFlags = 16384;  // T x R token-rank flags (bytes)
-constexpr int kSmallChunks = kSmallMaxPairs / kSmallThreads;  // 32-pair chunks per warp
-constexpr int kSmallMaxSmem = (kSmallWarps * kSmallMaxE + kSmallMaxE + 1 + kSmallMaxRE + kSmallMaxR) * 4 +
-                              kSmallMaxFlags;
+constexpr int kSmallMaxTileFlags = 8192;  // tile tokens x R flag bytes
+// pairs per CTA <= (T/C + 1) * k <= kSmallMaxPairs / C + kMaxK
+constexpr int kSmallChunks = ((kSmallMaxPairs / kClusterCtas + kMaxK) / kSmallWarps + kWarp - 1) / kWarp + 1;
+
+__host__ __device__ inline int small_tile_tokens(int T) { return (T + kClusterCtas - 1) / kClusterCtas; }
 
 __host__ __device__ inline bool layout_small_fits(int T, int k, int E, int R) {
   return static_cast<int64_t>(T) * k <= kSmallMaxPairs && E <= kSmallMaxE && R <= kSmallMaxR &&
-         R * E <= kSmallMaxRE && static_cast<int64_t>(T) * R <= kSmallMaxFlags;
+         R * E <= kSmallMaxRE && static_cast<int64_t>(small_tile_tokens(T)) * R <= kSmallMaxTileFlags;
 }
 
+// shared memory, int32 words then flag bytes:
+//   hist[E] base[E] whist[W][E] eoff[E+1] cnt[R*E] rank_cnt[R] flags[tile tokens * R]
 __host__ __device__ inline int layout_small_smem(int T, int E, int R) {
-  return (kSmallWarps * E + (E + 1) + R * E + R) * 4 + T * R;
+  return (2 * E + kSmallWarps * E + (E + 1) + R * E + R) * 4 + small_tile_tokens(T) * R;
 }
 
-__global__ void __launch_bounds__(kSmallThreads) layout_small_kernel(LayoutParams p) {
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSmallThreads)
+layout_small_kernel(LayoutParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ int32_t smem[];
-  int32_t* whist = smem;                          // [32][E]
-  int32_t* eoff = whist + kSmallWarps * p.E;      // [E + 1]
-  int32_t* cnt = eoff + p.E + 1;                  // [R][E] pairs by (source rank, expert)
-  int32_t* rank_cnt = cnt + p.R * p.E;            // [R]
-  uint8_t* flags = reinterpret_cast<uint8_t*>(rank_cnt + p.R);  // [T][R]
+  int32_t* hist = smem;                              // [E]   this tile's pairs per expert (read by all CTAs)
+  int32_t* base = hist + p.E;                        // [E]   pairs of each expert in earlier tiles
+  int32_t* whist = base + p.E;                       // [W][E]
+  int32_t* eoff = whist + kSmallWarps * p.E;         // [E + 1]
+  int32_t* cnt = eoff + p.E + 1;                     // [R][E] this tile's pairs by (source rank, expert)
+  int32_t* rank_cnt = cnt + p.R * p.E;               // [R]   this tile's tokens per destination rank
+  uint8_t* flags = reinterpret_cast<uint8_t*>(rank_cnt + p.R);  // [tile tokens][R]
   __shared__ int32_t scratch[kWarp];
+  const int c = static_cast<int>(cluster.block_rank());
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
-  const int P = p.T * p.k;
-  const int S = ((P + kSmallWarps - 1) / kSmallWarps + kWarp - 1) / kWarp * kWarp;
-  const int my_lo = warp * S, my_hi = min(my_lo + S, P);
+  const int t0 = static_cast<int>(static_cast<int64_t>(c) * p.T / kClusterCtas);
+  const int t1 = static_cast<int>(static_cast<int64_t>(c + 1) * p.T / kClusterCtas);
+  const int ntok = t1 - t0;
+  const int npairs = ntok * p.k;
+  const int64_t pair0 = static_cast<int64_t>(t0) * p.k;
+  const int S = ((npairs + kSmallWarps - 1) / kSmallWarps + kWarp - 1) / kWarp * kWarp;
+  const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
 
   bool bad = false;
   int ereg[kSmallChunks];
 #pragma unroll
-  for (int c = 0; c < kSmallChunks; ++c) {
-    const int i = my_lo + c * kWarp + lane;
-    ereg[c] = i < my_hi ? pair_expert(p, p.topk_idx[i], bad) : -1;
+  for (int q = 0; q < kSmallChunks; ++q) {
+    const int i = my_lo + q * kWarp + lane;
+    ereg[q] = i < my_hi ? pair_expert(p, p.topk_idx[pair0 + i], bad) : -1;
   }
-  for (int i = threadIdx.x; i < kSmallWarps * p.E; i += blockDim.x) whist[i] = 0;
-  for (int i = threadIdx.x; i < p.R * p.E + p.R; i += blockDim.x) cnt[i] = 0;  // cnt and rank_cnt
-  for (int i = threadIdx.x; i < p.T * p.R; i += blockDim.x) flags[i] = 0;
+  for (int i = threadIdx.x; i < (2 + kSmallWarps) * p.E; i += blockDim.x) hist[i] = 0;  // hist, base, whist
+  for (int i = threadIdx.x; i < p.R * p.E + p.R; i += blockDim.x) cnt[i] = 0;         // cnt, rank_cnt
+  for (int i = threadIdx.x; i < ntok * p.R; i += blockDim.x) flags[i] = 0;
   __syncthreads();
 
+  // ---- phase 1: count this tile
   int32_t* wh = whist + warp * p.E;
 #pragma unroll
-  for (int c = 0; c < kSmallChunks; ++c) {
-    const int i = my_lo + c * kWarp + lane;
-    const int e = ereg[c];
+  for (int q = 0; q < kSmallChunks; ++q) {
+    const int i = my_lo + q * kWarp + lane;
+    const int e = ereg[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
-    const int key = e >= 0 ? (i / p.k / p.Tr) * p.E + e : -1;
+    const int tl = e >= 0 ? i / p.k : 0;  // token within the tile
+    const int key = e >= 0 ? ((t0 + tl) / p.Tr) * p.E + e : -1;
     const unsigned same_key = __match_any_sync(0xffffffffu, key);
     if (key >= 0 && lane == __ffs(same_key) - 1) atomicAdd(&cnt[key], __popc(same_key));
-    if (e >= 0) flags[(i / p.k) * p.R + e / p.Er] = 1;
+    if (e >= 0) flags[tl * p.R + e / p.Er] = 1;
     __syncwarp();
   }
   __syncthreads();
-
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
     int32_t tot = 0;
     for (int w = 0; w < kSmallWarps; ++w) tot += whist[w * p.E + e];
+    hist[e] = tot;
+  }
+  for (int b0 = 0; b0 < ntok * p.R; b0 += blockDim.x) {  // uniform trip count
+    const int i = b0 + threadIdx.x;
+    const uint8_t f = i < ntok * p.R ? flags[i] : 0;
+    if (i < ntok * p.R) p.is_token_in_rank[static_cast<int64_t>(t0) * p.R + i] = f;
+    const int key = f ? i % p.R : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&rank_cnt[key], __popc(same));
+  }
+  cluster.sync();  // every tile's hist, cnt and rank_cnt are final
+
+  // ---- phase 2: totals and this tile's bases from every tile's histogram
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+    int32_t tot = 0, before = 0;
+#pragma unroll
+    for (int r = 0; r < kClusterCtas; ++r) {
+      const int32_t n = cluster.map_shared_rank(hist, r)[e];
+      before += r < c ? n : 0;
+      tot += n;
+    }
     eoff[e] = tot;
-    p.num_tokens_per_expert[e] = tot;
+    base[e] = before;
   }
   __syncthreads();
   const int32_t p_eff = block_exclusive_scan(eoff, p.E, scratch);
   if (threadIdx.x == 0) eoff[p.E] = p_eff;
   __syncthreads();
-  for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
-    p.expert_offset[e] = eoff[e];
-    if (e == p.E) break;
-    int32_t run = eoff[e];
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+    int32_t run = eoff[e] + base[e];
     for (int w = 0; w < kSmallWarps; ++w) {
       const int32_t n = whist[w * p.E + e];
       whist[w * p.E + e] = run;
       run += n;
     }
-    run = eoff[e];
-    for (int r = 0; r < p.R; ++r) {
-      const int32_t n = cnt[r * p.E + e];
-      p.src_rank_expert_offset[r * p.E + e] = run;
-      p.count_src_rank_expert[r * p.E + e] = n;
-      run += n;
-    }
   }
   __syncthreads();
-
   const uint32_t lt = lanemask_lt();
 #pragma unroll
-  for (int c = 0; c < kSmallChunks; ++c) {
-    const int i = my_lo + c * kWarp + lane;
-    const int e = ereg[c];
+  for (int q = 0; q < kSmallChunks; ++q) {
+    const int i = my_lo + q * kWarp + lane;
+    const int e = ereg[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
       const int32_t s = wh[e] + __popc(same & lt);
-      p.slot_of_pair[i] = s;
-      p.src_of_slot[s] = i;
+      p.slot_of_pair[pair0 + i] = s;
+      p.src_of_slot[s] = static_cast<int32_t>(pair0 + i);
     } else if (i < my_hi) {
-      p.slot_of_pair[i] = -1;
+      p.slot_of_pair[pair0 + i] = -1;
     }
     __syncwarp();
     if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
     __syncwarp();
   }
-  for (int i = p_eff + threadIdx.x; i < P; i += blockDim.x) p.src_of_slot[i] = -1;
 
-  // is_token_in_rank and per-rank token counts from the flags
-  for (int base = 0; base < p.T * p.R; base += blockDim.x) {  // uniform trip count
-    const int i = base + threadIdx.x;
-    const uint8_t f = i < p.T * p.R ? flags[i] : 0;
-    if (i < p.T * p.R) p.is_token_in_rank[i] = f;
-    const int key = f ? i % p.R : -1;
-    const unsigned same = __match_any_sync(0xffffffffu, key);
-    if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&rank_cnt[key], __popc(same));
+  // summaries, spread over the cluster
+  if (c == 0) {
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
+      p.expert_offset[e] = eoff[e];
+      if (e < p.E) p.num_tokens_per_expert[e] = eoff[e + 1] - eoff[e];
+    }
+    for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
+      int32_t n = 0;
+#pragma unroll
+      for (int q = 0; q < kClusterCtas; ++q) n += cluster.map_shared_rank(rank_cnt, q)[r];
+      p.num_tokens_per_rank[r] = n;
+    }
+  }
+  // per-(source rank, expert) totals: CTA c owns experts [e_lo, e_hi); one
+  // thread per (rank, owned expert) gathers the cluster's counts in one round
+  // of distributed-shared-memory loads, then one thread per expert walks the
+  // ranks for the offsets.  whist is free again after the ranking loop.
+  __syncthreads();
+  int32_t* tot_re = whist;  // [R][e_hi - e_lo]
+  const int e_lo = c * p.E / kClusterCtas, e_hi = (c + 1) * p.E / kClusterCtas, ne = e_hi - e_lo;
+  for (int i = threadIdx.x; i < p.R * ne; i += blockDim.x) {
+    const int r = i / ne, e = e_lo + (i - r * ne);
+    int32_t m = 0;
+#pragma unroll
+    for (int q = 0; q < kClusterCtas; ++q) m += cluster.map_shared_rank(cnt, q)[r * p.E + e];
+    tot_re[i] = m;
+    p.count_src_rank_expert[r * p.E + e] = m;
   }
   __syncthreads();
-  for (int r = threadIdx.x; r < p.R; r += blockDim.x) p.num_tokens_per_rank[r] = rank_cnt[r];
+  for (int el = threadIdx.x; el < ne; el += blockDim.x) {
+    int32_t run = eoff[e_lo + el];
+    for (int r = 0; r < p.R; ++r) {
+      p.src_rank_expert_offset[r * p.E + e_lo + el] = run;
+      run += tot_re[r * ne + el];
+    }
+  }
+  const int P = p.T * p.k;
+  for (int i = p_eff + c * blockDim.x + threadIdx.x; i < P; i += kClusterCtas * blockDim.x) p.src_of_slot[i] = -1;
   if (bad) atomicOr(p.error_word, 1);
+  cluster.sync();  // keep this CTA's shared memory until the others are done reading it
 }
 
 }  // namespace ep
