@@ -174,9 +174,9 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
 // its k receive rows by k TMA bulk copies (cp.async.bulk global <- shared)
 // issued by one thread, so every destination row is written as one
 // contiguous H- or 2H-byte transfer instead of 512-byte pieces from many
-// warps.  Two row stages alternate; before a stage is rewritten, the issuing
-// thread waits until the bulk copies of two tokens ago have finished reading
-// it (cp.async.bulk.wait_group.read).  The next token's x is loaded into
+// warps.  2 or 3 row stages rotate; before a stage is rewritten, the issuing
+// thread waits until the bulk copies that last read it have finished
+// (cp.async.bulk.wait_group.read).  The next token's x is loaded into
 // registers while the current one is quantised and stored.  Scales and gate
 // weights are written with plain stores from shared memory.
 
@@ -185,21 +185,33 @@ constexpr int kTmaMaxChunks = 16;
 
 struct TmaSmemLayout {
   int row_bytes;   // payload row bytes, rounded up to 128
+  int stages;      // payload row stages (2..3): as many as fit in kTmaRowBudget
   int off_slot;    // int32 [2][kMaxK]
   int off_w;       // float [2][kMaxK]
   int off_scale;   // float [2][G]
   int total;
 };
 
+constexpr int kTmaRowBudget = 40 * 1024;
+
 __host__ __device__ inline TmaSmemLayout tma_smem_layout(int H, bool fp8) {
   TmaSmemLayout L;
   const int row = fp8 ? H : 2 * H;
   L.row_bytes = (row + 127) / 128 * 128;
-  L.off_slot = 2 * L.row_bytes;
+  L.stages = kTmaRowBudget / L.row_bytes;
+  L.stages = L.stages < 2 ? 2 : (L.stages > 3 ? 3 : L.stages);
+  L.off_slot = L.stages * L.row_bytes;
   L.off_w = L.off_slot + 2 * kMaxK * 4;
   L.off_scale = L.off_w + 2 * kMaxK * 4;
   L.total = L.off_scale + (fp8 ? 2 * (H / kGroup) * 4 : 0);
   return L;
+}
+
+// Waits until at most stages-1 bulk-copy groups of this thread still read shared memory.
+__device__ __forceinline__ void bulk_wait_read_all_but(int n) {
+  if (n >= 3) asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
+  else if (n == 2) asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+  else asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 __device__ __forceinline__ void bulk_store_row(void* gdst, uint32_t ssrc, int bytes) {
@@ -227,7 +239,7 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
   }
   for (int it = 0; t < p.T; ++it, t += gridDim.x) {
     const int stage = it & 1;
-    uint8_t* row = tma_smem + stage * L.row_bytes;
+    uint8_t* row = tma_smem + (it % L.stages) * L.row_bytes;
     int32_t* sslot = reinterpret_cast<int32_t*>(tma_smem + L.off_slot) + stage * kMaxK;
     float* sw = reinterpret_cast<float*>(tma_smem + L.off_w) + stage * kMaxK;
     float* sscale = reinterpret_cast<float*>(tma_smem + L.off_scale) + stage * p.G;
@@ -240,8 +252,8 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
       if (a0) n0 = ld_ro_v4(xr);
       if (a1) n1 = ld_ro_v4(xr + 8);
     }
-    // the row stage is free once the copies issued two tokens ago have read it
-    if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    // the row stage is free once the copies issued L.stages tokens ago have read it
+    if (threadIdx.x == 0) bulk_wait_read_all_but(L.stages - 1);
     if (warp == 0 && lane < p.k) {
       sslot[lane] = p.slot_of_pair[static_cast<int64_t>(t) * p.k + lane];
       sw[lane] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];

@@ -19,7 +19,7 @@ import numpy as np
 
 from . import build as _build
 
-OK, BAD_INDEX, INVALID = 0, 1, 2
+OK, BAD_INDEX, INVALID, CAPACITY = 0, 1, 2, 4
 
 _lib = None
 
@@ -44,6 +44,8 @@ def lib():
             f.argtypes = [p, i64, p]
         L.epo_layout.restype = ctypes.c_int
         L.epo_layout.argtypes = [i64, i64, i64, i64] + [p] * 9
+        L.epo_layout_padded.restype = ctypes.c_int
+        L.epo_layout_padded.argtypes = [i64, i64, i64, i64, i64] + [p] * 9
         L.epo_dispatch_bf16.restype = None
         L.epo_dispatch_bf16.argtypes = [i64, i64, i64] + [p] * 5
         L.epo_dispatch_fp8.restype = None
@@ -121,6 +123,33 @@ def layout(topk_idx: np.ndarray, E: int, R: int) -> dict:
                                                  "slot_of_pair", "src_of_slot")))
     if st == INVALID:
         raise ValueError("oracle layout: invalid shape")
+    d["status"] = st
+    return d
+
+
+def layout_padded(topk_idx: np.ndarray, E: int, R: int, M: int) -> dict:
+    """Padded (low-latency) layout: receive rows [E][R][M]; returns the handle
+    arrays ("src_of_slot" has E*R*M entries) plus ``status`` (bit flags
+    BAD_INDEX | CAPACITY, or OK)."""
+    idx = _c(topk_idx, np.int64)
+    T, k = idx.shape
+    d = {
+        "num_tokens_per_expert": np.zeros(E, np.int32),
+        "expert_offset": np.zeros(E + 1, np.int32),
+        "num_tokens_per_rank": np.zeros(R, np.int32),
+        "count_src_rank_expert": np.zeros(R * E, np.int32),
+        "src_rank_expert_offset": np.zeros(R * E, np.int32),
+        "is_token_in_rank": np.zeros(T * R, np.uint8),
+        "slot_of_pair": np.zeros(T * k, np.int32),
+        "src_of_slot": np.zeros(E * R * M, np.int32),
+    }
+    st = lib().epo_layout_padded(T, k, E, R, M, _ptr(idx),
+                                 *(_ptr(d[n]) for n in ("num_tokens_per_expert", "expert_offset",
+                                                        "num_tokens_per_rank", "count_src_rank_expert",
+                                                        "src_rank_expert_offset", "is_token_in_rank",
+                                                        "slot_of_pair", "src_of_slot")))
+    if st == INVALID:
+        raise ValueError("oracle padded layout: invalid shape")
     d["status"] = st
     return d
 

@@ -176,6 +176,50 @@ int epo_layout(int64_t T, int64_t k, int64_t E, int64_t R, const int64_t* topk_i
   return status;
 }
 
+/* Padded layout (the low-latency kernels' static receive buffer: per local
+ * expert, R blocks of M rows, one block per source rank). */
+int epo_layout_padded(int64_t T, int64_t k, int64_t E, int64_t R, int64_t M, const int64_t* topk_idx,
+                      int32_t* num_tokens_per_expert, int32_t* expert_offset,
+                      int32_t* num_tokens_per_rank, int32_t* count_src_rank_expert,
+                      int32_t* src_rank_expert_offset, uint8_t* is_token_in_rank,
+                      int32_t* slot_of_pair, int32_t* src_of_row) {
+  if (T < 0 || k < 1 || E < 1 || R < 1 || E % R != 0 || T % R != 0 || M < T / R || M < 1) return EPO_INVALID;
+  int64_t Tr = T / R, Er = E / R;
+  int status = EPO_OK;
+
+  for (int64_t e = 0; e < E; ++e) num_tokens_per_expert[e] = 0;
+  for (int64_t i = 0; i < R * E; ++i) count_src_rank_expert[i] = 0;
+  for (int64_t i = 0; i < T * R; ++i) is_token_in_rank[i] = 0;
+  for (int64_t i = 0; i < E * R * M; ++i) src_of_row[i] = -1;
+  for (int64_t e = 0; e <= E; ++e) expert_offset[e] = (int32_t)(e * R * M);
+  for (int64_t r = 0; r < R; ++r)
+    for (int64_t e = 0; e < E; ++e) src_rank_expert_offset[r * E + e] = (int32_t)((e * R + r) * M);
+
+  /* walk the pairs in (t, j) order; (source rank, expert) blocks fill in turn */
+  for (int64_t t = 0; t < T; ++t) {
+    int64_t r = t / Tr;
+    for (int64_t j = 0; j < k; ++j) {
+      int64_t e = topk_idx[t * k + j];
+      slot_of_pair[t * k + j] = -1;
+      if (e == -1) continue;
+      if (e < -1 || e >= E) { status |= EPO_BAD_INDEX; continue; }
+      num_tokens_per_expert[e] += 1;
+      is_token_in_rank[t * R + e / Er] = 1;
+      int64_t i = count_src_rank_expert[r * E + e]++;
+      if (i >= M) { status |= EPO_CAPACITY; continue; }
+      int64_t row = (e * R + r) * M + i;
+      slot_of_pair[t * k + j] = (int32_t)row;
+      src_of_row[row] = (int32_t)(t * k + j);
+    }
+  }
+  for (int64_t r = 0; r < R; ++r) {
+    int32_t n = 0;
+    for (int64_t t = 0; t < T; ++t) n += is_token_in_rank[t * R + r];
+    num_tokens_per_rank[r] = n;
+  }
+  return status;
+}
+
 /* --------------------------------------------------------------- dispatch */
 
 void epo_dispatch_bf16(int64_t T, int64_t H, int64_t k, const uint16_t* x,

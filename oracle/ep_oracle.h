@@ -22,6 +22,7 @@
 #define EPO_OK 0
 #define EPO_BAD_INDEX 1
 #define EPO_INVALID 2
+#define EPO_CAPACITY 4  /* padded layout: a pair beyond max_tokens_per_rank (bit, may combine with BAD_INDEX) */
 
 #ifdef __cplusplus
 extern "C" {
@@ -43,6 +44,17 @@ int epo_layout(int64_t T, int64_t k, int64_t E, int64_t R, const int64_t* topk_i
                int32_t* num_tokens_per_rank, int32_t* count_src_rank_expert,
                int32_t* src_rank_expert_offset, uint8_t* is_token_in_rank,
                int32_t* slot_of_pair, int32_t* src_of_slot);
+
+/* Padded ("low-latency") layout: receive rows [E][R][M]; pair (t, j) with
+ * expert e from source rank r = t / (T/R) takes row (e*R + r)*M + i, i its
+ * position among rank r's pairs to e in (t, j) order.  i >= M: no row,
+ * EPO_CAPACITY.  src_of_row has E*R*M entries, -1 where no pair landed.
+ * expert_offset[e] = e*R*M, src_rank_expert_offset[r*E+e] = (e*R+r)*M. */
+int epo_layout_padded(int64_t T, int64_t k, int64_t E, int64_t R, int64_t M, const int64_t* topk_idx,
+                      int32_t* num_tokens_per_expert, int32_t* expert_offset,
+                      int32_t* num_tokens_per_rank, int32_t* count_src_rank_expert,
+                      int32_t* src_rank_expert_offset, uint8_t* is_token_in_rank,
+                      int32_t* slot_of_pair, int32_t* src_of_row);
 
 void epo_dispatch_bf16(int64_t T, int64_t H, int64_t k, const uint16_t* x,
                        const float* topk_weights, const int32_t* slot_of_pair,

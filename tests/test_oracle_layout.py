@@ -133,3 +133,85 @@ def test_workload_invariants(name):
     bounds = offs[np.arange(0, w.E + 1, Er)]
     assert bounds[0] == 0 and bounds[-1] == P and np.all(np.diff(bounds) >= 0)
     assert_layout_equal(got, sort_based_layout(idx, w.E, w.R))
+
+
+# ----------------------------------------------------- padded (low-latency) layout
+
+def sort_based_padded(idx, E, R, M):
+    """Padded rows as a sort: valid pairs stably sorted by block key e*R + r
+    (pairs are in (t, j) order before); a pair's position in its block is its
+    sorted index minus the block's first index."""
+    T, k = idx.shape
+    Tr = T // R
+    flat = idx.reshape(-1)
+    valid = (flat >= 0) & (flat < E)
+    tok = np.repeat(np.arange(T), k)
+    key = np.where(valid, flat * R + tok // max(Tr, 1), E * R)
+    order = np.argsort(key, kind="stable")
+    skey = key[order]
+    first = np.searchsorted(skey, skey, side="left")
+    pos = np.arange(order.size) - first
+    slot = np.full(T * k, -1, np.int64)
+    ok = (skey < E * R) & (pos < M)
+    slot[order[ok]] = skey[ok] * M + pos[ok]
+    rows = np.full(E * R * M, -1, np.int64)
+    rows[slot[slot >= 0]] = np.nonzero(slot >= 0)[0]
+    overflow = bool(np.any((skey < E * R) & (pos >= M)))
+    return slot, rows, overflow
+
+
+@pytest.mark.parametrize("T,k,E,R", [(2, 2, 2, 1), (2, 2, 2, 2), (3, 2, 3, 1), (4, 1, 4, 2)])
+def test_padded_brute_force_all_tables(T, k, E, R):
+    Tr = T // R
+    for M in (Tr, Tr + 1):
+        for entries in itertools.product(range(-1, E), repeat=T * k):
+            idx = np.array(entries, np.int64).reshape(T, k)
+            got = oracle.layout_padded(idx, E, R, M)
+            slot, rows, overflow = sort_based_padded(idx, E, R, M)
+            assert np.array_equal(got["slot_of_pair"], slot)
+            assert np.array_equal(got["src_of_slot"], rows)
+            assert bool(got["status"] & oracle.CAPACITY) == overflow
+            dense = oracle.layout(idx, E, R)
+            for n in ("num_tokens_per_expert", "num_tokens_per_rank", "count_src_rank_expert",
+                      "is_token_in_rank"):
+                assert np.array_equal(got[n], dense[n]), n
+            assert np.array_equal(got["expert_offset"], np.arange(E + 1) * R * M)
+
+
+def test_padded_random_tables_and_capacity():
+    rng = np.random.default_rng(21)
+    for trial in range(100):
+        R = int(rng.integers(1, 5))
+        E = R * int(rng.integers(1, 5))
+        T = R * int(rng.integers(1, 7))
+        k = int(rng.integers(1, 5))
+        M = T // R + int(rng.integers(0, 3))
+        idx = rng.integers(-1, E, size=(T, k)).astype(np.int64)  # duplicates allowed
+        got = oracle.layout_padded(idx, E, R, M)
+        slot, rows, overflow = sort_based_padded(idx, E, R, M)
+        assert np.array_equal(got["slot_of_pair"], slot)
+        assert np.array_equal(got["src_of_slot"], rows)
+        assert bool(got["status"] & oracle.CAPACITY) == overflow
+    with pytest.raises(ValueError):
+        oracle.layout_padded(np.zeros((8, 2), np.int64), 4, 2, 3)  # M < T/R
+
+
+def test_padded_decode_workload_invariants():
+    w = wl.CONFIGS["decode"]
+    idx, _, _ = wl.routing(w)
+    M = w.T // w.R
+    got = oracle.layout_padded(idx, w.E, w.R, M)
+    assert got["status"] == oracle.OK  # distinct experts per token: never over capacity
+    slots = got["slot_of_pair"]
+    flat = idx.reshape(-1)
+    r_of_pair = np.repeat(np.arange(w.T), w.k) // M
+    block = slots // M
+    assert np.array_equal(block, flat * w.R + r_of_pair)  # each pair in its (expert, source rank) block
+    assert np.array_equal(got["src_of_slot"][slots], np.arange(w.T * w.k))
+    pos = slots % M
+    cnt = got["count_src_rank_expert"].reshape(w.R, w.E)
+    assert np.all(pos < cnt[r_of_pair, flat])  # rows packed from the block start
+    # same rank-relative positions as the dense layout
+    dense = oracle.layout(idx, w.E, w.R)
+    rel_dense = dense["slot_of_pair"] - dense["src_rank_expert_offset"].reshape(w.R, w.E)[r_of_pair, flat]
+    assert np.array_equal(pos, rel_dense)

@@ -56,6 +56,10 @@ MUTATIONS = [
      "      run += count_src_rank_expert[r * E + e];\n      src_rank_expert_offset[r * E + e] = run;", "test_oracle_layout.py"),
     ("bad ids not flagged", "if (e < -1 || e >= E) { status = EPO_BAD_INDEX; continue; }",
      "if (e < -1 || e >= E) { continue; }", "test_oracle_layout.py"),
+    ("padded blocks rank-major", "int64_t row = (e * R + r) * M + i;", "int64_t row = (r * E + e) * M + i;",
+     "test_oracle_layout.py"),
+    ("padded overflow not flagged", "if (i >= M) { status |= EPO_CAPACITY; continue; }",
+     "if (i >= M) { continue; }", "test_oracle_layout.py"),
 ]
 
 
@@ -106,4 +110,4 @@ def test_pins_reject_every_mutant(tmp_path):
         results = list(ex.map(check, range(len(MUTATIONS))))
     survived = [(name, out) for name, rc, out in results if rc == 0]
     assert not survived, "the pins accepted: " + "; ".join(n for n, _ in survived)
-    assert len(results) == len(MUTATIONS) >= 15
+    assert len(results) == len(MUTATIONS) >= 19
