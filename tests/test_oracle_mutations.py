@@ -50,7 +50,9 @@ MUTATIONS = [
      "  for (int64_t t = 0; t < T; ++t) {\n    for (int64_t j = 0; j < k; ++j) {\n      int64_t e = topk_idx[t * k + j];\n      if (e < 0 || e >= E) { slot_of_pair",
      "  for (int64_t j = 0; j < k; ++j) {\n    for (int64_t t = 0; t < T; ++t) {\n      int64_t e = topk_idx[t * k + j];\n      if (e < 0 || e >= E) { slot_of_pair",
      "test_oracle_layout.py"),
-    ("rank of an expert by modulo", "is_token_in_rank[t * R + e / Er] = 1;", "is_token_in_rank[t * R + e % R] = 1;",
+    ("rank of an expert by modulo",
+     "is_token_in_rank[t * R + e / Er] = 1;\n      count_src_rank_expert[(t / Tr) * E + e] += 1;",
+     "is_token_in_rank[t * R + e % R] = 1;\n      count_src_rank_expert[(t / Tr) * E + e] += 1;",
      "test_oracle_layout.py"),
     ("source-rank offsets one rank late", "      src_rank_expert_offset[r * E + e] = run;\n      run += count_src_rank_expert[r * E + e];",
      "      run += count_src_rank_expert[r * E + e];\n      src_rank_expert_offset[r * E + e] = run;", "test_oracle_layout.py"),
