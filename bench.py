@@ -185,12 +185,13 @@ class ClockSampler:
 class Path:
     """Device buffers of one workload and one step through the C ABI."""
 
-    def __init__(self, w, d, dev):
+    def __init__(self, w, d, dev, max_tokens_per_rank=0):
         import numpy as np
         import torch
         import combine_ep_get_histogram_b200 as ep
         self.ep, self.w, self.dev = ep, w, dev
-        P = w.T * w.k
+        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8, 0, max_tokens_per_rank)
+        P = ep.ep.receive_rows(self.shape)
 
         def bf16(a):
             return torch.from_numpy(a.view(np.int16))
@@ -198,7 +199,6 @@ class Path:
         self.host = {"topk_idx": torch.from_numpy(d["topk_idx"]), "topk_weights": torch.from_numpy(d["topk_weights"]),
                      "x": bf16(d["x"]), "y": bf16(d["y"]), "g": bf16(d["g"])}
         self.inp = {n: t.to(dev) for n, t in self.host.items()}
-        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8)
         self.handle = ep.Handle(self.shape, dev)
         self.ws = ep.workspace(self.shape, dev)
         self.recv_x = torch.empty((P, w.H), dtype=torch.uint8 if w.use_fp8 else torch.int16, device=dev)
@@ -244,8 +244,11 @@ def run_ours(args, rank, world, local):
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     w = workload(args)
-    d = wl.make_inputs(w, parts=("routing", "x", "y", "g"))
-    path = Path(w, d, dev)
+    M = args.max_tokens_per_rank
+    d = wl.make_inputs(w, parts=("routing", "x", "g") + (() if M else ("y",)))
+    if M:  # expert outputs fill the padded receive rows
+        d["y"] = wl.normal_bf16(w.E * w.R * M, w.H, w.seed, 2)
+    path = Path(w, d, dev, M)
     stream = torch.cuda.current_stream()
     nb = call_bytes(w)
     step_bytes = sum(nb.values())
@@ -373,6 +376,8 @@ def run_ours(args, rank, world, local):
                                f"{'FP8' if w.use_fp8 else 'BF16'} dispatch + BF16 combine + both backward passes",
                    "T": w.T, "H": w.H, "k": w.k, "E": w.E, "R": w.R, "use_fp8": w.use_fp8,
                    "step_bytes": step_bytes, "l2": "inputs larger than L2 (no flush)",
+                   "receive_layout": (f"padded [E][R][{args.max_tokens_per_rank}]" if args.max_tokens_per_rank
+                                      else "dense [T*k]"),
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, virtual ranks"},
         "per_call": per_call,
         "roofline": {"kernel": kernel_of[dominant], "call": dominant, "bound": "hbm", "achieved": ach,
@@ -455,6 +460,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--max-tokens-per-rank", type=int, default=0,
+                    help="padded low-latency receive layout with this many rows per (expert, source rank)")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="resize the workload to R x this many tokens (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -68,6 +68,8 @@ int device_info(const DeviceInfo** out) {
     d.sms = prop.multiProcessorCount;
     d.supported = prop.major == 10 && prop.minor == 0;
     if (d.supported) {
+      cudaFuncSetAttribute(reinterpret_cast<const void*>(layout_padded_kernel),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kPadMaxSmem);
       d.occ_count = occupancy(reinterpret_cast<const void*>(layout_count_kernel), kLayoutThreads,
                               (kMaxE + kMaxR) * 4 + kTileFlagBytes);
       d.occ_disp_bf16 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<false>), kMoveThreads, 0);
@@ -97,7 +99,19 @@ int check_shape(const ep_shape_t* s) {
   if (s->use_fp8 && s->H % kGroup != 0) return EP_ERR_INVALID_ARG;
   if (s->num_sms < 0) return EP_ERR_INVALID_ARG;
   if (static_cast<int64_t>(s->T) * s->k > 0x7fffffffLL) return EP_ERR_INVALID_ARG;
+  if (s->max_tokens_per_rank < 0) return EP_ERR_INVALID_ARG;
+  if (s->max_tokens_per_rank > 0) {  // padded low-latency layout
+    const int64_t Tr = s->T / s->R, M = s->max_tokens_per_rank;
+    if (M < Tr || static_cast<int64_t>(s->E) * s->R * M > 0x7fffffffLL || Tr * s->k > kPadMaxPairs ||
+        Tr * s->R > kPadMaxFlags)
+      return EP_ERR_INVALID_ARG;
+  }
   return EP_OK;
+}
+
+int64_t receive_rows(const ep_shape_t* s) {
+  return s->max_tokens_per_rank > 0 ? static_cast<int64_t>(s->E) * s->R * s->max_tokens_per_rank
+                                    : static_cast<int64_t>(s->T) * s->k;
 }
 
 int check_handle(const ep_shape_t* s, const ep_handle_t* h) {
@@ -175,7 +189,7 @@ int ep_handle_sizes(const ep_shape_t* shape, int64_t counts[9]) {
   int st = check_shape(shape);
   if (st != EP_OK || counts == nullptr) return EP_ERR_INVALID_ARG;
   const int64_t T = shape->T, k = shape->k, E = shape->E, R = shape->R;
-  const int64_t c[9] = {E, E + 1, R, R * E, R * E, T * R, T * k, T * k, 1};
+  const int64_t c[9] = {E, E + 1, R, R * E, R * E, T * R, T * k, receive_rows(shape), 1};
   for (int i = 0; i < 9; ++i) counts[i] = c[i];
   return EP_OK;
 }
@@ -222,6 +236,14 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
   p.error_word = handle->error_word;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (shape->max_tokens_per_rank > 0) {
+    if ((st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_expert, 0, shape->E * 4, s))) != EP_OK ||
+        (st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_rank, 0, shape->R * 4, s))) != EP_OK)
+      return st;
+    layout_padded_kernel<<<shape->R, kPadThreads, layout_padded_smem(p.Tr, shape->E, shape->R), s>>>(
+        p, shape->max_tokens_per_rank);
+    return finish(handle, s);
+  }
   if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
     layout_small_kernel<<<kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s>>>(p);
     return finish(handle, s);
@@ -350,7 +372,8 @@ int ep_get_error(const ep_handle_t* handle, ep_stream_t stream) {
     return st;
   if ((st = cuda_status(cudaMemsetAsync(handle->error_word, 0, 4, s))) != EP_OK) return st;
   if ((st = cuda_status(cudaStreamSynchronize(s))) != EP_OK) return st;
-  return (word & 1) ? EP_ERR_BAD_INDEX : EP_OK;
+  if (word & 1) return EP_ERR_BAD_INDEX;
+  return (word & 2) ? EP_ERR_CAPACITY : EP_OK;
 }
 
 const char* ep_status_string(int status) {
@@ -363,6 +386,8 @@ const char* ep_status_string(int status) {
     case EP_ERR_SCRATCH_TOO_SMALL:
       return "EP_ERR_SCRATCH_TOO_SMALL: the shape needs more layout scratch than the no-alloc entry point's "
              "fixed array holds (ep_noalloc_scratch_bytes)";
+    case EP_ERR_CAPACITY:
+      return "EP_ERR_CAPACITY: a padded (source rank, expert) block received more than max_tokens_per_rank pairs";
     default: return "unknown ep status";
   }
 }

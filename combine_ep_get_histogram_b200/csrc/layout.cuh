@@ -460,4 +460,123 @@ layout_small_kernel(LayoutParams p) {
   cluster.sync();  // keep this CTA's shared memory until the others are done reading it
 }
 
+// ------------------------------------------------ padded low-latency layout
+//
+// Receive rows [E][R][M]: the pairs of (source rank r, expert e) fill block
+// (e*R + r) from its first row in (t, j) order.  No block depends on another
+// source rank, so one CTA per source rank does the whole layout in one
+// launch: per-warp expert histograms of the rank's pairs (contiguous runs),
+// an exclusive scan over warps per expert from 0, ranking with
+// popc(same_expert_mask & lanemask_lt).  Totals over ranks
+// (num_tokens_per_expert, num_tokens_per_rank) are integer atomics into
+// arrays zeroed just before the launch, so their values do not depend on
+// order.  Rows a block does not fill are marked -1 in src_of_slot.
+
+constexpr int kPadThreads = 512;
+constexpr int kPadWarps = kPadThreads / kWarp;
+constexpr int kPadMaxPairs = 8192;   // pairs of one source rank
+constexpr int kPadMaxFlags = 32768;  // (T/R) x R token-rank flag bytes
+constexpr int kPadChunks = (kPadMaxPairs / kPadWarps + kWarp - 1) / kWarp;  // 16
+
+__host__ __device__ inline int layout_padded_smem(int Tr, int E, int R) {
+  return (kPadWarps * E + E + R) * 4 + Tr * R;  // whist[W][E] cnt[E] rank_cnt[R] flags[Tr][R]
+}
+constexpr int kPadMaxSmem = (kPadWarps * kMaxE + kMaxE + kMaxR) * 4 + kPadMaxFlags;
+
+__global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams p, int M) {
+  extern __shared__ int32_t smem[];
+  int32_t* whist = smem;                         // [W][E]
+  int32_t* cnt = whist + kPadWarps * p.E;        // [E] this rank's pairs per expert
+  int32_t* rank_cnt = cnt + p.E;                 // [R] this rank's tokens per destination rank
+  uint8_t* flags = reinterpret_cast<uint8_t*>(rank_cnt + p.R);  // [Tr][R]
+  const int r = blockIdx.x;
+  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
+  const int npairs = p.Tr * p.k;
+  const int64_t pair0 = static_cast<int64_t>(r) * p.Tr * p.k;
+  const int S = ((npairs + kPadWarps - 1) / kPadWarps + kWarp - 1) / kWarp * kWarp;
+  const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
+
+  bool bad = false, over = false;
+  int ereg[kPadChunks];
+#pragma unroll
+  for (int q = 0; q < kPadChunks; ++q) {
+    const int i = my_lo + q * kWarp + lane;
+    ereg[q] = i < my_hi ? pair_expert(p, p.topk_idx[pair0 + i], bad) : -1;
+  }
+  for (int i = threadIdx.x; i < (kPadWarps + 1) * p.E + p.R; i += blockDim.x) whist[i] = 0;  // whist, cnt, rank_cnt
+  for (int i = threadIdx.x; i < p.Tr * p.R; i += blockDim.x) flags[i] = 0;
+  __syncthreads();
+
+  int32_t* wh = whist + warp * p.E;
+#pragma unroll
+  for (int q = 0; q < kPadChunks; ++q) {
+    const int i = my_lo + q * kWarp + lane;
+    const int e = ereg[q];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
+    if (e >= 0) flags[(i / p.k) * p.R + e / p.Er] = 1;
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < kPadWarps; ++w) {
+      const int32_t n = whist[w * p.E + e];
+      whist[w * p.E + e] = run;
+      run += n;
+    }
+    cnt[e] = run;
+    p.count_src_rank_expert[r * p.E + e] = run;
+    p.src_rank_expert_offset[r * p.E + e] = (e * p.R + r) * M;
+    if (run > 0) atomicAdd(&p.num_tokens_per_expert[e], run);
+  }
+  if (r == 0)
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.expert_offset[e] = e * p.R * M;
+  __syncthreads();
+
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int q = 0; q < kPadChunks; ++q) {
+    const int i = my_lo + q * kWarp + lane;
+    const int e = ereg[q];
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    if (e >= 0) {
+      const int32_t pos = wh[e] + __popc(same & lt);
+      if (pos < M) {
+        const int32_t row = (e * p.R + r) * M + pos;
+        p.slot_of_pair[pair0 + i] = row;
+        p.src_of_slot[row] = static_cast<int32_t>(pair0 + i);
+      } else {
+        p.slot_of_pair[pair0 + i] = -1;
+        over = true;
+      }
+    } else if (i < my_hi) {
+      p.slot_of_pair[pair0 + i] = -1;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
+    __syncwarp();
+  }
+  // rows of this rank's blocks that no pair filled
+  for (int64_t q = threadIdx.x; q < static_cast<int64_t>(p.E) * M; q += blockDim.x) {
+    const int e = static_cast<int>(q / M), i = static_cast<int>(q - static_cast<int64_t>(e) * M);
+    if (i >= cnt[e]) p.src_of_slot[static_cast<int64_t>(e * p.R + r) * M + i] = -1;
+  }
+  // is_token_in_rank and token counts per destination rank
+  uint8_t* itr = p.is_token_in_rank + static_cast<int64_t>(r) * p.Tr * p.R;
+  for (int b0 = 0; b0 < p.Tr * p.R; b0 += blockDim.x) {  // uniform trip count
+    const int i = b0 + threadIdx.x;
+    const uint8_t f = i < p.Tr * p.R ? flags[i] : 0;
+    if (i < p.Tr * p.R) itr[i] = f;
+    const int key = f ? i % p.R : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&rank_cnt[key], __popc(same));
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < p.R; d += blockDim.x)
+    if (rank_cnt[d] > 0) atomicAdd(&p.num_tokens_per_rank[d], rank_cnt[d]);
+  if (bad) atomicOr(p.error_word, 1);
+  if (over) atomicOr(p.error_word, 2);
+}
+
 }  // namespace ep

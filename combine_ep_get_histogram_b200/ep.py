@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libep_b200.
 
 EP_OK, EP_ERR_INVALID_ARG, EP_ERR_BAD_INDEX, EP_ERR_CUDA, EP_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
 EP_ERR_SCRATCH_TOO_SMALL = 5
+EP_ERR_CAPACITY = 6
 
 HANDLE_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank",
                  "count_src_rank_expert", "src_rank_expert_offset", "is_token_in_rank",
@@ -33,7 +34,8 @@ EXPORTED = ("ep_handle_sizes", "ep_workspace_size", "ep_get_dispatch_layout", "e
 
 
 class ep_shape_t(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("T", "H", "k", "E", "R", "use_fp8", "num_sms")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "H", "k", "E", "R", "use_fp8", "num_sms",
+                                              "max_tokens_per_rank")]
 
 
 class ep_handle_t(ctypes.Structure):
@@ -113,8 +115,16 @@ def _check(status: int, where: str) -> int:
     return status
 
 
-def make_shape(T: int, H: int, k: int, E: int, R: int, use_fp8: bool = False, num_sms: int = 0) -> ep_shape_t:
-    return ep_shape_t(T, H, k, E, R, int(bool(use_fp8)), num_sms)
+def make_shape(T: int, H: int, k: int, E: int, R: int, use_fp8: bool = False, num_sms: int = 0,
+               max_tokens_per_rank: int = 0) -> ep_shape_t:
+    """max_tokens_per_rank = 0: dense receive layout (T*k rows); M > 0: padded
+    low-latency layout (E*R*M rows, see include/ep.h)."""
+    return ep_shape_t(T, H, k, E, R, int(bool(use_fp8)), num_sms, max_tokens_per_rank)
+
+
+def receive_rows(shape: ep_shape_t) -> int:
+    M = shape.max_tokens_per_rank
+    return shape.E * shape.R * M if M > 0 else shape.T * shape.k
 
 
 def handle_sizes(shape: ep_shape_t) -> dict:

@@ -22,8 +22,12 @@
  *
  * Model of the expert-parallel world: one GPU, R virtual ranks.  Rank r owns
  * source tokens [r*T/R, (r+1)*T/R) and experts [r*E/R, (r+1)*E/R).  Every
- * receive buffer is one array of P = T*k rows in expert-major order; rank r's
- * partition is rows [expert_offset[r*E/R], expert_offset[(r+1)*E/R]).
+ * receive buffer is one array of rows in expert-major order; rank r's
+ * partition is rows [expert_offset[r*E/R], expert_offset[(r+1)*E/R]).  Dense
+ * layout: P = T*k rows, no gaps.  Padded layout (the low-latency kernels'
+ * static per-expert buffers, sized by num_max_tokens_per_rank, for decoding
+ * with CUDA graphs: blog.hotdry.top, sections 一 and 二; zhouruolin.cn,
+ * section 五): E*R*M rows, see ep_shape_t.max_tokens_per_rank.
  *
  * Numerics (the pages do not fix them; these are the definitions used):
  *  - slots: the pairs routed to expert e take rows [expert_offset[e],
@@ -57,7 +61,8 @@
  *    found on the device: the pair is treated as masked and bit 0 of
  *    handle->error_word is set; ep_get_error reports it.
  *  - Limits: 0 <= T, T % R == 0, 1 <= k <= 32, 1 <= E <= 1024, 1 <= R <= E,
- *    E % R == 0, T*k < 2^31, 8 <= H, H % 8 == 0 (H % 128 == 0 with FP8).
+ *    E % R == 0, T*k < 2^31, 8 <= H, H % 8 == 0 (H % 128 == 0 with FP8);
+ *    padded layout: see max_tokens_per_rank.
  */
 #ifndef EP_B200_H
 #define EP_B200_H
@@ -78,8 +83,10 @@ typedef enum {
   EP_ERR_BAD_INDEX = 2,    /* a topk_idx entry outside [-1, E) (from ep_get_error) */
   EP_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
   EP_ERR_UNSUPPORTED = 4,  /* the current device is not an sm_100 GPU */
-  EP_ERR_SCRATCH_TOO_SMALL = 5 /* the shape needs more layout scratch than
-                                  ep_get_dispatch_layout_noalloc's fixed array */
+  EP_ERR_SCRATCH_TOO_SMALL = 5, /* the shape needs more layout scratch than
+                                   ep_get_dispatch_layout_noalloc's fixed array */
+  EP_ERR_CAPACITY = 6           /* padded layout: some (source rank, expert) block got more
+                                   than max_tokens_per_rank pairs (from ep_get_error) */
 } ep_status_t;
 
 /* Problem shape. T tokens over R virtual ranks, hidden H, top-k, E experts. */
@@ -88,6 +95,15 @@ typedef struct {
   int32_t use_fp8; /* 1: dispatch writes E4M3 codes + fp32 scales; 0: bf16 rows */
   int32_t num_sms; /* SMs a call may fill: 0 = all.  Caps each grid at
                       num_sms x (resident CTAs per SM). */
+  int32_t max_tokens_per_rank; /* 0: dense receive layout (below).  M > 0:
+                      the padded low-latency layout: E*R*M receive rows, one
+                      block of M rows per (expert e, source rank r) at row
+                      (e*R + r)*M; the pair (t, j) takes row (e*R + r)*M + i,
+                      i its position among rank r's pairs to e in (t, j)
+                      order.  Needs M >= T/R, E*R*M < 2^31, (T/R)*k <= 8192.
+                      Pairs past M get no row (EP_ERR_CAPACITY via
+                      ep_get_error; only duplicate experts in a row can cause
+                      it).  Rows with no pair are not written. */
 } ep_shape_t;
 
 /* The dispatch handle: device arrays written by ep_get_dispatch_layout and
@@ -96,11 +112,12 @@ typedef struct {
   int32_t* num_tokens_per_expert;  /* [E]   pairs routed to each expert */
   int32_t* expert_offset;          /* [E+1] exclusive prefix sum of the above */
   int32_t* num_tokens_per_rank;    /* [R]   tokens with >= 1 pair on rank r */
-  int32_t* count_src_rank_expert;  /* [R*E] pairs from source rank r to expert e */
+  int32_t* count_src_rank_expert;  /* [R*E] pairs from source rank r to expert e (padded: may exceed M) */
   int32_t* src_rank_expert_offset; /* [R*E] first row of (source rank r, expert e) */
   uint8_t* is_token_in_rank;       /* [T*R] 1 if token t has a pair on rank r */
   int32_t* slot_of_pair;           /* [T*k] receive row of pair (t,j); -1 if masked */
-  int32_t* src_of_slot;            /* [T*k] t*k+j of the pair in each row; -1 past the last row */
+  int32_t* src_of_slot;            /* [rows] t*k+j of the pair in each receive row, -1 if none;
+                                      rows = T*k (dense) or E*R*M (padded) */
   int32_t* error_word;             /* [1]   device error bits; must be 0 before first use */
 } ep_handle_t;
 
@@ -170,8 +187,9 @@ int ep_get_dispatch_layout_noalloc(const ep_shape_t* shape, const int64_t* topk_
 size_t ep_noalloc_scratch_bytes(void);
 
 /* Synchronises `stream`, reads handle->error_word, clears it, and returns
- * EP_ERR_BAD_INDEX if a bad expert id was seen since the last call, EP_OK if
- * not, EP_ERR_CUDA if the stream reports an error. */
+ * EP_ERR_BAD_INDEX if a bad expert id was seen since the last read, else
+ * EP_ERR_CAPACITY if a padded block overflowed, else EP_OK; EP_ERR_CUDA if
+ * the stream reports an error. */
 int ep_get_error(const ep_handle_t* handle, ep_stream_t stream);
 
 /* Static description of a status code. */

@@ -27,11 +27,12 @@ class GpuPath:
     """One workload on the GPU: the handle, the layout and the buffers."""
 
     def __init__(self, w, topk_idx: np.ndarray, topk_weights: np.ndarray, device,
-                 use_fp8: bool | None = None, num_sms: int = 0):
+                 use_fp8: bool | None = None, num_sms: int = 0, max_tokens_per_rank: int = 0):
         self.w = w
         self.device = device
         self.use_fp8 = w.use_fp8 if use_fp8 is None else use_fp8
-        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, self.use_fp8, num_sms)
+        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, self.use_fp8, num_sms, max_tokens_per_rank)
+        self.rows = ep.ep.receive_rows(self.shape)
         self.handle = ep.Handle(self.shape, device)
         self.ws = ep.workspace(self.shape, device)
         self.idx = to_dev(topk_idx, device)
@@ -50,7 +51,7 @@ class GpuPath:
 
     def dispatch(self, x_dev, fill=0):
         w = self.w
-        P = w.T * w.k
+        P = self.rows
         if self.use_fp8:
             recv_x = torch.full((max(P, 1), w.H), fill, dtype=torch.uint8, device=self.device)
             recv_scale = torch.full((max(P, 1), w.H // 128), float(fill), dtype=torch.float32,
@@ -69,7 +70,7 @@ class GpuPath:
 
     def combine_backward(self, g_dev, y_dev):
         w = self.w
-        grad_y = torch.zeros((max(w.T * w.k, 1), w.H), dtype=torch.int16, device=self.device)
+        grad_y = torch.zeros((max(self.rows, 1), w.H), dtype=torch.int16, device=self.device)
         grad_w = torch.full((max(w.T, 1), w.k), -7.0, dtype=torch.float32, device=self.device)
         ep.ep_combine_backward(self.shape, g_dev, y_dev, self.wts, self.handle, grad_y, grad_w)
         return grad_y, grad_w

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for st in range(6):
+    for st in range(7):
         assert binding.status_string(st).startswith("EP_")
 
 

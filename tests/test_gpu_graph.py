@@ -17,10 +17,10 @@ pytestmark = pytest.mark.gpu
 
 
 class Step:
-    def __init__(self, w, device):
+    def __init__(self, w, device, max_tokens_per_rank=0):
         self.w = w
-        P = w.T * w.k
-        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8)
+        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8, 0, max_tokens_per_rank)
+        P = ep.ep.receive_rows(self.shape)
         self.h = ep.Handle(self.shape, device)
         self.ws = ep.workspace(self.shape, device)
         self.idx = torch.empty((w.T, w.k), dtype=torch.int64, device=device)
@@ -51,7 +51,7 @@ class Step:
 
     def outputs(self):
         torch.cuda.synchronize()
-        n = int(self.h.expert_offset[-1].item())
+        n = self.rx.shape[0] if self.shape.max_tokens_per_rank else int(self.h.expert_offset[-1].item())
         res = [self.h.tensors[f].clone() for f in ("slot_of_pair", "src_of_slot", "expert_offset",
                                                     "num_tokens_per_rank", "is_token_in_rank")]
         res += [self.rx[:n].clone(), self.rw[:n].clone(), self.out.clone(), self.gy[:n].clone(),
@@ -61,20 +61,24 @@ class Step:
         return res
 
 
-@pytest.mark.parametrize("name", ["decode", "tiny"])
-def test_step_replays_from_a_cuda_graph(cuda_device, name):
+@pytest.mark.parametrize("name,padded", [("decode", False), ("tiny", False), ("tiny", True)])
+def test_step_replays_from_a_cuda_graph(cuda_device, name, padded):
     w = wl.CONFIGS[name]
+    M = w.T // w.R if padded else 0
     inputs = [wl.make_inputs(w.with_(seed=s), parts=("routing", "x", "y", "g")) for s in (0, 1)]
+    if padded:  # expert outputs live in the padded receive rows
+        for s, d in enumerate(inputs):
+            d["y"] = wl.normal_bf16(w.E * w.R * M, w.H, s, 2)
     assert not np.array_equal(inputs[0]["topk_idx"], inputs[1]["topk_idx"])
 
-    eager = Step(w, cuda_device)
+    eager = Step(w, cuda_device, M)
     expected = []
     for d in inputs:
         eager.load(d)
         eager.run()
         expected.append(eager.outputs())
 
-    step = Step(w, cuda_device)
+    step = Step(w, cuda_device, M)
     step.load(inputs[0])
     step.run()  # first use on the device happens outside the capture
     torch.cuda.synchronize()
