@@ -46,6 +46,8 @@ def lib():
         L.epo_layout.argtypes = [i64, i64, i64, i64] + [p] * 9
         L.epo_layout_padded.restype = ctypes.c_int
         L.epo_layout_padded.argtypes = [i64, i64, i64, i64, i64] + [p] * 9
+        L.epo_route_group_limited.restype = ctypes.c_int
+        L.epo_route_group_limited.argtypes = [i64, i64, i64, i64, i64, p, p, p]
         L.epo_dispatch_bf16.restype = None
         L.epo_dispatch_bf16.argtypes = [i64, i64, i64] + [p] * 5
         L.epo_dispatch_fp8.restype = None
@@ -152,6 +154,17 @@ def layout_padded(topk_idx: np.ndarray, E: int, R: int, M: int) -> dict:
         raise ValueError("oracle padded layout: invalid shape")
     d["status"] = st
     return d
+
+
+def route_group_limited(scores: np.ndarray, k: int, n_groups: int, topk_groups: int):
+    """scores [T,E] float32 -> (topk_idx [T,k] int64, topk_weights [T,k] float32)."""
+    sc = _c(scores, np.float32)
+    T, E = sc.shape
+    idx = np.zeros((T, k), np.int64)
+    w = np.zeros((T, k), np.float32)
+    if lib().epo_route_group_limited(T, E, k, n_groups, topk_groups, _ptr(sc), _ptr(idx), _ptr(w)) == INVALID:
+        raise ValueError("oracle routing: invalid arguments")
+    return idx, w
 
 
 # ------------------------------------------------------------ data movement

@@ -220,6 +220,57 @@ int epo_layout_padded(int64_t T, int64_t k, int64_t E, int64_t R, int64_t M, con
   return status;
 }
 
+/* ---------------------------------------------------------------- routing */
+
+/* Group-limited gating: experts are split into groups and a token first
+ * chooses groups, then experts inside them ("top-4 groups, top-8 experts":
+ * blog.hotdry.top section 一 and section 三 on group-limited gating). */
+int epo_route_group_limited(int64_t T, int64_t E, int64_t k, int64_t n_groups, int64_t topk_groups,
+                            const float* scores, int64_t* topk_idx, float* topk_weights) {
+  if (n_groups < 1 || E % n_groups != 0 || topk_groups < 1 || topk_groups > n_groups) return EPO_INVALID;
+  int64_t per = E / n_groups;
+  if (k < 1 || k > topk_groups * per) return EPO_INVALID;
+  float* gscore = (float*)malloc((size_t)n_groups * sizeof(float));
+  char* gsel = (char*)malloc((size_t)n_groups);
+  char* taken = (char*)malloc((size_t)E);
+  for (int64_t t = 0; t < T; ++t) {
+    const float* s = scores + t * E;
+    for (int64_t g = 0; g < n_groups; ++g) {
+      float m = s[g * per];
+      for (int64_t i = 1; i < per; ++i)
+        if (s[g * per + i] > m) m = s[g * per + i];
+      gscore[g] = m;
+      gsel[g] = 0;
+    }
+    /* best groups: repeatedly the highest remaining group score, lowest index on ties */
+    for (int64_t n = 0; n < topk_groups; ++n) {
+      int64_t best = -1;
+      for (int64_t g = 0; g < n_groups; ++g)
+        if (!gsel[g] && (best < 0 || gscore[g] > gscore[best])) best = g;
+      gsel[best] = 1;
+    }
+    /* best experts inside the chosen groups, in order */
+    for (int64_t e = 0; e < E; ++e) taken[e] = 0;
+    for (int64_t j = 0; j < k; ++j) {
+      int64_t best = -1;
+      for (int64_t e = 0; e < E; ++e)
+        if (gsel[e / per] && !taken[e] && (best < 0 || s[e] > s[best])) best = e;
+      taken[best] = 1;
+      topk_idx[t * k + j] = best;
+    }
+    /* softmax of the chosen scores */
+    double mx = s[topk_idx[t * k]], sum = 0.0;
+    for (int64_t j = 1; j < k; ++j)
+      if (s[topk_idx[t * k + j]] > mx) mx = s[topk_idx[t * k + j]];
+    for (int64_t j = 0; j < k; ++j) sum += exp((double)s[topk_idx[t * k + j]] - mx);
+    for (int64_t j = 0; j < k; ++j) topk_weights[t * k + j] = (float)(exp((double)s[topk_idx[t * k + j]] - mx) / sum);
+  }
+  free(gscore);
+  free(gsel);
+  free(taken);
+  return EPO_OK;
+}
+
 /* --------------------------------------------------------------- dispatch */
 
 void epo_dispatch_bf16(int64_t T, int64_t H, int64_t k, const uint16_t* x,

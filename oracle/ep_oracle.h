@@ -56,6 +56,14 @@ int epo_layout_padded(int64_t T, int64_t k, int64_t E, int64_t R, int64_t M, con
                       int32_t* src_rank_expert_offset, uint8_t* is_token_in_rank,
                       int32_t* slot_of_pair, int32_t* src_of_row);
 
+/* Group-limited top-k routing of scores [T,E] (E experts in n_groups groups of
+ * E/n_groups consecutive experts): group score = max of its experts' scores;
+ * the topk_groups best groups are kept, then the k best experts inside them.
+ * Ties go to the lower index.  topk_idx lists the experts by descending score;
+ * topk_weights = softmax of their scores (computed in double). */
+int epo_route_group_limited(int64_t T, int64_t E, int64_t k, int64_t n_groups, int64_t topk_groups,
+                            const float* scores, int64_t* topk_idx, float* topk_weights);
+
 void epo_dispatch_bf16(int64_t T, int64_t H, int64_t k, const uint16_t* x,
                        const float* topk_weights, const int32_t* slot_of_pair,
                        uint16_t* recv_x, float* recv_weight);

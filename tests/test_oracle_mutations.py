@@ -62,6 +62,12 @@ MUTATIONS = [
      "test_oracle_layout.py"),
     ("padded overflow not flagged", "if (i >= M) { status |= EPO_CAPACITY; continue; }",
      "if (i >= M) { continue; }", "test_oracle_layout.py"),
+    ("router group ties to the higher index", "if (!gsel[g] && (best < 0 || gscore[g] > gscore[best])) best = g;",
+     "if (!gsel[g] && (best < 0 || gscore[g] >= gscore[best])) best = g;", "test_oracle_router.py"),
+    ("router ignores the group limit", "if (gsel[e / per] && !taken[e] && (best < 0 || s[e] > s[best])) best = e;",
+     "if (!taken[e] && (best < 0 || s[e] > s[best])) best = e;", "test_oracle_router.py"),
+    ("router group score is the first expert", "if (s[g * per + i] > m) m = s[g * per + i];",
+     "if (0) m = s[g * per + i];", "test_oracle_router.py"),
 ]
 
 
@@ -92,7 +98,7 @@ def run_pins(lib, test_file):
 
 def test_unmodified_copy_passes(tmp_path):
     lib = build_variant(tmp_path, "unmodified")
-    for f in ("test_oracle_formats.py", "test_oracle_ops.py", "test_oracle_layout.py"):
+    for f in ("test_oracle_formats.py", "test_oracle_ops.py", "test_oracle_layout.py", "test_oracle_router.py"):
         rc, out = run_pins(lib, f)
         assert rc == 0, out
 
