@@ -37,6 +37,7 @@ if ROOT not in sys.path:
 
 METRIC = "dispatch/combine µs/call & effective GB/s vs B200 roofline, 1 GPU"
 CALLS = ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward")
+ROUTE_CALLS = ("route",) + CALLS
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -45,6 +46,7 @@ def call_bytes(w) -> dict:
     T, H, k, R = w.T, w.H, w.k, w.R
     disp = T * H * 2 + (T * k * (H + 4 * (H // 128)) if w.use_fp8 else T * k * H * 2)
     return {
+        "route": T * w.E * 4 + T * k * (8 + 4),
         "layout": T * k * 8 + T * R + 2 * T * k * 4,
         "dispatch": disp,
         "combine": T * k * H * 2 + T * k * 4 + T * H * 2,
@@ -185,7 +187,7 @@ class ClockSampler:
 class Path:
     """Device buffers of one workload and one step through the C ABI."""
 
-    def __init__(self, w, d, dev, max_tokens_per_rank=0):
+    def __init__(self, w, d, dev, max_tokens_per_rank=0, route=False):
         import numpy as np
         import torch
         import combine_ep_get_histogram_b200 as ep
@@ -198,6 +200,9 @@ class Path:
 
         self.host = {"topk_idx": torch.from_numpy(d["topk_idx"]), "topk_weights": torch.from_numpy(d["topk_weights"]),
                      "x": bf16(d["x"]), "y": bf16(d["y"]), "g": bf16(d["g"])}
+        self.route = route
+        if route:
+            self.host["scores"] = torch.from_numpy(d["scores"])
         self.inp = {n: t.to(dev) for n, t in self.host.items()}
         self.handle = ep.Handle(self.shape, dev)
         self.ws = ep.workspace(self.shape, dev)
@@ -211,20 +216,31 @@ class Path:
 
     def step(self, marks=None):
         ep, i = self.ep, self.inp
-        rec = (lambda n: marks[n].record()) if marks is not None else (lambda n: None)
-        rec(0)
+        n = 0
+
+        def rec():
+            nonlocal n
+            if marks is not None:
+                marks[n].record()
+            n += 1
+
+        rec()
+        if self.route:
+            ep.ep_route_group_limited(self.shape, i["scores"], self.w.n_groups, self.w.topk_groups, i["topk_idx"],
+                                      i["topk_weights"])
+            rec()
         ep.ep_get_dispatch_layout(self.shape, i["topk_idx"], self.handle, self.ws)
-        rec(1)
+        rec()
         ep.ep_dispatch(self.shape, i["x"], i["topk_weights"], self.handle, self.recv_x, self.recv_scale,
                        self.recv_weight)
-        rec(2)
+        rec()
         ep.ep_combine(self.shape, i["y"], i["topk_weights"], self.handle, self.out)
-        rec(3)
+        rec()
         ep.ep_combine_backward(self.shape, i["g"], i["y"], i["topk_weights"], self.handle, self.grad_y,
                                self.grad_w)
-        rec(4)
+        rec()
         ep.ep_dispatch_backward(self.shape, self.grad_y, self.handle, self.grad_x)
-        rec(5)
+        rec()
 
 
 def launches_per_step(w) -> int:
@@ -245,13 +261,15 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(dev)
     w = workload(args)
     M = args.max_tokens_per_rank
-    d = wl.make_inputs(w, parts=("routing", "x", "g") + (() if M else ("y",)))
+    calls = ROUTE_CALLS if args.route else CALLS
+    d = wl.make_inputs(w, parts=("routing", "x", "g") + (() if M else ("y",)) + (("scores",) if args.route else ()))
     if M:  # expert outputs fill the padded receive rows
         d["y"] = wl.normal_bf16(w.E * w.R * M, w.H, w.seed, 2)
-    path = Path(w, d, dev, M)
+    path = Path(w, d, dev, M, route=args.route)
     stream = torch.cuda.current_stream()
-    nb = call_bytes(w)
+    nb = {c: v for c, v in call_bytes(w).items() if c in calls}
     step_bytes = sum(nb.values())
+    nmarks = len(calls) + 1
 
     def barrier():
         torch.cuda.synchronize()
@@ -265,11 +283,11 @@ def run_ours(args, rank, world, local):
     # One step is captured as a CUDA graph (the C ABI never allocates or
     # synchronises), so small workloads are not timed against Python's call
     # overhead; events recorded inside the graph mark the call boundaries.
-    per_call_ms = {c: [] for c in CALLS}
+    per_call_ms = {c: [] for c in calls}
     if args.no_graph:
         run_step = path.step
     else:
-        gmarks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+        gmarks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nmarks)]
         graph = torch.cuda.CUDAGraph()
         torch.cuda.synchronize()
         with torch.cuda.graph(graph):
@@ -281,12 +299,12 @@ def run_ours(args, rank, world, local):
         for _ in range(min(args.steps, 20)):
             run_step()
             torch.cuda.synchronize()
-            for ci, c in enumerate(CALLS):
+            for ci, c in enumerate(calls):
                 per_call_ms[c].append(gmarks[ci].elapsed_time(gmarks[ci + 1]))
         barrier()
 
     # device-timed region: K steps back to back on the launching stream
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(nmarks)] for _ in range(args.steps)]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     sampler.start()
@@ -306,7 +324,7 @@ def run_ours(args, rank, world, local):
     clocks = sampler.stop()
     if args.no_graph:
         for m in marks:
-            for ci, c in enumerate(CALLS):
+            for ci, c in enumerate(calls):
                 per_call_ms[c].append(m[ci].elapsed_time(m[ci + 1]))
     total_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
     ms_per_step = total_ms / args.steps
@@ -348,15 +366,16 @@ def run_ours(args, rank, world, local):
 
     peak, peak_kind = peaks()
     per_call = {}
-    for c in CALLS:
+    for c in calls:
         us = 1e3 * statistics.mean(per_call_ms[c])
         per_call[c] = {"us": round(us, 2), "us_median": round(1e3 * statistics.median(per_call_ms[c]), 2),
                        "bytes": nb[c], "GB_s": round(nb[c] / (us * 1e-6) / 1e9, 1),
                        "frac_of_peak": round(nb[c] / (us * 1e-6) / 1e9 / peak, 3)}
-    dominant = max((c for c in CALLS), key=lambda c: per_call[c]["us"])
+    dominant = max((c for c in calls), key=lambda c: per_call[c]["us"])
     kernel_of = {"dispatch": "dispatch_tma_kernel<FP8>" if w.use_fp8 else "dispatch_tma_kernel<BF16>",
                  "combine": "gather_reduce_kernel<weighted>", "combine_backward": "combine_backward_kernel",
-                 "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel"}
+                 "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel",
+                 "route": "route_group_limited_kernel"}
     ach = per_call[dominant]["GB_s"]
     line = {
         "metric": METRIC,
@@ -386,7 +405,7 @@ def run_ours(args, rank, world, local):
                      "bytes_per_launch": nb[dominant], "traffic": measured_traffic(w, dominant),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, full-size launch"},
         "clocks": clocks,
-        "gpu_launches": launches_per_step(w) * args.steps,
+        "gpu_launches": (launches_per_step(w) + (1 if args.route else 0)) * args.steps,
         "timing": "CUDA graph replay of the step" if not args.no_graph else "eager launches",
         "e2e": e2e,
     }
@@ -460,6 +479,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--route", action="store_true",
+                    help="start each step with group-limited routing of [T,E] scores (the step before the path)")
     ap.add_argument("--max-tokens-per-rank", type=int, default=0,
                     help="padded low-latency receive layout with this many rows per (expert, source rank)")
     ap.add_argument("--tokens-per-rank", type=int, default=0,

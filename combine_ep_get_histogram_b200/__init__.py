@@ -10,5 +10,5 @@ from . import workloads  # noqa: F401  (inputs only; no method arithmetic)
 from .ep import (  # noqa: F401
     EPError, Handle, make_shape, workspace, workspace_size, handle_sizes, library,
     ep_get_dispatch_layout, ep_get_dispatch_layout_noalloc, ep_dispatch, ep_combine, ep_combine_backward,
-    ep_dispatch_backward, ep_get_error,
+    ep_dispatch_backward, ep_get_error, ep_route_group_limited,
 )

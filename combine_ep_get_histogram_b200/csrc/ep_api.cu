@@ -11,6 +11,7 @@
 #include "ep.h"
 #include "layout.cuh"
 #include "movement.cuh"
+#include "route.cuh"
 
 namespace {
 
@@ -41,6 +42,7 @@ struct DeviceInfo {
   int occ_disp_bf16 = 0, occ_disp_fp8 = 0, occ_comb = 0, occ_dbwd = 0;
   int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
   int occ_cbwd = 0;
+  int occ_route[6] = {};  // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
 };
 
 constexpr int kMaxDevices = 64;
@@ -77,6 +79,13 @@ int device_info(const DeviceInfo** out) {
       d.occ_comb = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<true>), kMoveThreads, 0);
       d.occ_dbwd = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false>), kMoveThreads, 0);
       d.occ_cbwd = occupancy(reinterpret_cast<const void*>(combine_backward_kernel), kMoveThreads, 0);
+      const void* route_fns[6] = {reinterpret_cast<const void*>(route_group_limited_kernel<1>),
+                                  reinterpret_cast<const void*>(route_group_limited_kernel<2>),
+                                  reinterpret_cast<const void*>(route_group_limited_kernel<4>),
+                                  reinterpret_cast<const void*>(route_group_limited_kernel<8>),
+                                  reinterpret_cast<const void*>(route_group_limited_kernel<16>),
+                                  reinterpret_cast<const void*>(route_group_limited_kernel<32>)};
+      for (int i = 0; i < 6; ++i) d.occ_route[i] = occupancy(route_fns[i], kRouteThreads, 0);
       cudaGetLastError();
     }
     g_dev[dev] = d;
@@ -360,6 +369,38 @@ int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv, const e
   gather_reduce_kernel<false><<<movement_grid(*d, shape, d->occ_dbwd, T * p.chunks), kMoveThreads, 0, s>>>(
       p, static_cast<const uint16_t*>(grad_recv), static_cast<uint16_t*>(grad_x));
   return finish(handle, s);
+}
+
+int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_groups, int topk_groups,
+                           int64_t* topk_idx, float* topk_weights, ep_stream_t stream) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if (n_groups < 1 || n_groups > kRouteMaxGroups || shape->E % n_groups != 0 || topk_groups < 1 ||
+      topk_groups > n_groups || shape->k > topk_groups * (shape->E / n_groups))
+    return EP_ERR_INVALID_ARG;
+  const int64_t T = shape->T;
+  if (T > 0 && (!f32_ok(scores, T) || topk_idx == nullptr || !aligned(topk_idx, 8) || !f32_ok(topk_weights, T)))
+    return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (T == 0) return EP_OK;
+  RouteParams p{scores, shape->T, shape->E, shape->k, n_groups, topk_groups, topk_idx, topk_weights};
+  constexpr int warps = kRouteThreads / kWarp;
+  const int nq = static_cast<int>(ceil_div(shape->E, kWarp));
+  const int variant = nq <= 1 ? 0 : nq <= 2 ? 1 : nq <= 4 ? 2 : nq <= 8 ? 3 : nq <= 16 ? 4 : 5;
+  const int64_t cap = grid_cap(*d, shape, d->occ_route[variant]);
+  const int64_t need = ceil_div(T, warps);
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (variant) {
+    case 0: route_group_limited_kernel<1><<<grid, kRouteThreads, 0, s>>>(p); break;
+    case 1: route_group_limited_kernel<2><<<grid, kRouteThreads, 0, s>>>(p); break;
+    case 2: route_group_limited_kernel<4><<<grid, kRouteThreads, 0, s>>>(p); break;
+    case 3: route_group_limited_kernel<8><<<grid, kRouteThreads, 0, s>>>(p); break;
+    case 4: route_group_limited_kernel<16><<<grid, kRouteThreads, 0, s>>>(p); break;
+    default: route_group_limited_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
+  }
+  return cuda_status(cudaGetLastError());
 }
 
 int ep_get_error(const ep_handle_t* handle, ep_stream_t stream) {

@@ -557,10 +557,10 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
     if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
     __syncwarp();
   }
-  // rows of this rank's blocks that no pair filled
-  for (int64_t q = threadIdx.x; q < static_cast<int64_t>(p.E) * M; q += blockDim.x) {
-    const int e = static_cast<int>(q / M), i = static_cast<int>(q - static_cast<int64_t>(e) * M);
-    if (i >= cnt[e]) p.src_of_slot[static_cast<int64_t>(e * p.R + r) * M + i] = -1;
+  // rows of this rank's blocks that no pair filled: one warp per expert block
+  for (int e = warp; e < p.E; e += kPadWarps) {
+    int32_t* blk = p.src_of_slot + static_cast<int64_t>(e * p.R + r) * M;
+    for (int i = min(cnt[e], M) + lane; i < M; i += kWarp) blk[i] = -1;
   }
   // is_token_in_rank and token counts per destination rank
   uint8_t* itr = p.is_token_in_rank + static_cast<int64_t>(r) * p.Tr * p.R;

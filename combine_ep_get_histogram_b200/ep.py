@@ -30,7 +30,7 @@ HANDLE_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank"
 EXPORTED = ("ep_handle_sizes", "ep_workspace_size", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_combine_backward", "ep_dispatch_backward", "ep_get_error",
             "ep_status_string", "ep_last_cuda_error", "ep_get_dispatch_layout_noalloc",
-            "ep_noalloc_scratch_bytes")
+            "ep_noalloc_scratch_bytes", "ep_route_group_limited")
 
 
 class ep_shape_t(ctypes.Structure):
@@ -75,6 +75,7 @@ def _lib():
             "ep_last_cuda_error": (ctypes.c_char_p, []),
             "ep_get_dispatch_layout_noalloc": (ctypes.c_int, [shp, vp, hp, vp]),
             "ep_noalloc_scratch_bytes": (ctypes.c_size_t, []),
+            "ep_route_group_limited": (ctypes.c_int, [shp, vp, ctypes.c_int, ctypes.c_int, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -206,6 +207,13 @@ def ep_dispatch_backward(shape: ep_shape_t, grad_recv, handle: Handle, grad_x, s
     st = _lib().ep_dispatch_backward(ctypes.byref(shape), _ptr(grad_recv), ctypes.byref(handle.c),
                                      _ptr(grad_x), _stream(stream))
     return _check(st, "ep_dispatch_backward") if check else st
+
+
+def ep_route_group_limited(shape: ep_shape_t, scores, n_groups: int, topk_groups: int, topk_idx, topk_weights,
+                           stream=None, check=True) -> int:
+    st = _lib().ep_route_group_limited(ctypes.byref(shape), _ptr(scores), n_groups, topk_groups, _ptr(topk_idx),
+                                       _ptr(topk_weights), _stream(stream))
+    return _check(st, "ep_route_group_limited") if check else st
 
 
 def ep_get_error(handle: Handle, stream=None) -> int:

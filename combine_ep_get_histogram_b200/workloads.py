@@ -19,6 +19,7 @@ in for real router traces.
 Draw recipe (seed 0 unless stated):
   * stream 0, one sequential ``numpy.random.default_rng([seed, 0])``:
     routing draws, then gate logits, then the outlier channel choice;
+  * stream 4: router scores [T, E], one float32 N(0, 1) draw;
   * streams 1 (x), 2 (expert outputs y) and 3 (grad_out g): row chunks of
     ``max(1, 2**22 // H)`` rows, chunk c drawn from
     ``default_rng([seed, stream, c])`` as float32 N(0, 1), multiplied by the
@@ -186,7 +187,8 @@ def make_inputs(w: Workload, parts=("routing", "x")) -> dict:
     """Draws the requested parts of a workload's inputs.
 
     parts: any of "routing" (topk_idx, topk_weights), "x" ([T,H] tokens),
-    "y" ([T*k,H] expert outputs), "g" ([T,H] grad of the combined output).
+    "y" ([T*k,H] expert outputs), "g" ([T,H] grad of the combined output),
+    "scores" ([T,E] float32 N(0,1) router scores, stream 4).
     """
     d: dict = {"workload": w}
     idx, wts, outliers = routing(w)
@@ -204,4 +206,8 @@ def make_inputs(w: Workload, parts=("routing", "x")) -> dict:
         d["y"] = normal_bf16(w.P, w.H, w.seed, 2, 1.0)
     if "g" in parts:
         d["g"] = normal_bf16(w.T, w.H, w.seed, 3, w.g_sigma)
+    if "scores" in parts:
+        sc = np.empty((w.T, w.E), dtype=np.float32)
+        np.random.default_rng([w.seed, 4]).standard_normal(out=sc, dtype=np.float32)
+        d["scores"] = sc
     return d

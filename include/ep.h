@@ -186,6 +186,19 @@ int ep_get_dispatch_layout_noalloc(const ep_shape_t* shape, const int64_t* topk_
 /* Size in bytes of ep_get_dispatch_layout_noalloc's fixed scratch array. */
 size_t ep_noalloc_scratch_bytes(void);
 
+/* Group-limited top-k routing, the step that produces topk_idx and
+ * topk_weights (experts split into groups; a token picks its best groups,
+ * then its top-k experts inside them: blog.hotdry.top "deepep-expert-
+ * parallel-communication-library", sections 一 and 三).
+ * scores: [T,E] fp32, finite, device.  Experts are n_groups groups of E /
+ * n_groups consecutive ids (n_groups <= 32); a group's score is its largest
+ * expert score; the topk_groups best groups are kept, then the k best
+ * experts inside them, ties to the lower index.  topk_idx [T,k] int64 lists
+ * them by descending score; topk_weights [T,k] fp32 = softmax of their
+ * scores.  Needs k <= topk_groups * E / n_groups.  One warp per token. */
+int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_groups, int topk_groups,
+                           int64_t* topk_idx, float* topk_weights, ep_stream_t stream);
+
 /* Synchronises `stream`, reads handle->error_word, clears it, and returns
  * EP_ERR_BAD_INDEX if a bad expert id was seen since the last read, else
  * EP_ERR_CAPACITY if a padded block overflowed, else EP_OK; EP_ERR_CUDA if

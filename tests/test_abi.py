@@ -112,3 +112,10 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_LIB", None)
     with pytest.raises(RuntimeError, match="not built"):
         binding.library()
+
+
+@pytest.mark.parametrize("ng,tg,k", [(0, 1, 2), (3, 2, 2), (8, 9, 2), (8, 2, 17), (64, 4, 2)])
+def test_route_bad_arguments_rejected_on_host(ng, tg, k):
+    s = ep.make_shape(T=64, H=128, k=k, E=64, R=4)
+    fake = 1 << 20
+    assert ep.library().ep_route_group_limited(ctypes.byref(s), fake, ng, tg, fake, fake, None) == 1

@@ -50,14 +50,19 @@ class Step:
         ep.ep_dispatch_backward(self.shape, self.gy, self.h, self.gx)
 
     def outputs(self):
+        """Handle arrays, and the receive rows that hold a pair (padded
+        layouts leave the other rows unwritten)."""
         torch.cuda.synchronize()
-        n = self.rx.shape[0] if self.shape.max_tokens_per_rank else int(self.h.expert_offset[-1].item())
+        if self.shape.max_tokens_per_rank:
+            rows = torch.nonzero(self.h.src_of_slot >= 0).squeeze(1)
+        else:
+            rows = torch.arange(int(self.h.expert_offset[-1].item()), device=self.rx.device)
         res = [self.h.tensors[f].clone() for f in ("slot_of_pair", "src_of_slot", "expert_offset",
                                                     "num_tokens_per_rank", "is_token_in_rank")]
-        res += [self.rx[:n].clone(), self.rw[:n].clone(), self.out.clone(), self.gy[:n].clone(),
+        res += [self.rx[rows].clone(), self.rw[rows].clone(), self.out.clone(), self.gy[rows].clone(),
                 self.gw.clone(), self.gx.clone()]
         if self.rs is not None:
-            res.append(self.rs[:n].clone())
+            res.append(self.rs[rows].clone())
         return res
 
 

@@ -1,0 +1,72 @@
+"""Group-limited top-k routing on the GPU against the oracle.
+
+The selections compare input scores only, so topk_idx must match exactly
+(ties included: many scores are quantised to force them); the weights are
+an fp32 softmax on the GPU against float64 in the oracle (2e-6 relative)."""
+
+import numpy as np
+import pytest
+import torch
+
+import combine_ep_get_histogram_b200 as ep
+import oracle
+from gpu_util import assert_layout_equal
+
+pytestmark = pytest.mark.gpu
+
+
+def scores_for(T, E, seed, ties=True):
+    rng = np.random.default_rng(seed)
+    s = rng.standard_normal((T, E)).astype(np.float32)
+    if ties:
+        s[: T // 2] = np.round(s[: T // 2] * 4) / 4  # exact ties in half the tokens
+    return s
+
+
+def route_gpu(device, s, k, ng, tg, R=1):
+    T, E = s.shape
+    shape = ep.make_shape(T, 128, k, E, R)
+    idx = torch.full((max(T, 1), k), -9, dtype=torch.int64, device=device)
+    w = torch.full((max(T, 1), k), -9.0, dtype=torch.float32, device=device)
+    ep.ep_route_group_limited(shape, torch.from_numpy(s).to(device), ng, tg, idx, w)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy()[:T], w.cpu().numpy()[:T]
+
+
+@pytest.mark.parametrize("T,E,k,ng,tg", [
+    (1024, 256, 8, 8, 4),      # decode shape: top-4 of 8 groups, top-8 experts
+    (32768, 256, 8, 8, 4),     # prefill shape
+    (512, 1024, 32, 32, 16),   # E and k at their maxima, 32 groups
+    (300, 48, 6, 3, 2),        # E not a multiple of 32, 16 experts per group
+    (200, 64, 5, 1, 1),        # one group: plain top-k
+    (100, 16, 16, 4, 4),       # every expert chosen
+])
+def test_route_matches_oracle(cuda_device, T, E, k, ng, tg):
+    s = scores_for(T, E, seed=T + E + k)
+    idx, w = route_gpu(cuda_device, s, k, ng, tg)
+    ridx, rw = oracle.route_group_limited(s, k, ng, tg)
+    assert np.array_equal(idx, ridx)
+    assert np.allclose(w, rw, rtol=2e-6, atol=0)
+
+
+def test_route_then_layout(cuda_device):
+    """Routing feeds the layout: the whole front of the path on the GPU
+    against oracle routing followed by the oracle layout."""
+    T, E, k, ng, tg, R = 2048, 256, 8, 8, 4, 8
+    s = scores_for(T, E, seed=5, ties=False)
+    shape = ep.make_shape(T, 128, k, E, R)
+    idx = torch.empty((T, k), dtype=torch.int64, device=cuda_device)
+    w = torch.empty((T, k), dtype=torch.float32, device=cuda_device)
+    ep.ep_route_group_limited(shape, torch.from_numpy(s).to(cuda_device), ng, tg, idx, w)
+    h = ep.Handle(shape, cuda_device)
+    ep.ep_get_dispatch_layout(shape, idx, h, ep.workspace(shape, cuda_device))
+    torch.cuda.synchronize()
+    ridx, _ = oracle.route_group_limited(s, k, ng, tg)
+    ref = oracle.layout(ridx, E, R)
+    got = {n: h.tensors[n].cpu().numpy()[: ep.handle_sizes(shape)[n]] for n in ref if n != "status"}
+    assert_layout_equal(got, {n: v for n, v in ref.items() if n != "status"})
+
+
+def test_route_empty(cuda_device):
+    idx, w = route_gpu(cuda_device, np.zeros((0, 64), np.float32), 4, 4, 2)
+    assert idx.shape == (0, 4)
