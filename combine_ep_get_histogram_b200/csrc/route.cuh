@@ -9,11 +9,14 @@
 // score with ties to the lower index; topk_idx lists the experts by
 // descending score; the weights are the softmax of the chosen scores.
 //
-// One warp per token.  Lane l holds the scores of experts l + 32q (coalesced
-// 128-byte loads).  Group maxima are warp reductions; groups, then experts,
-// are picked by repeated warp arg-max over (score, lower index first).  The
-// selections compare input scores only, so they are exact; the softmax uses
-// fp32 expf.  Scores must be finite.
+// One warp per token.  Lane l holds the scores of the contiguous experts
+// [l*NQ, (l+1)*NQ), so lane order is expert order.  Scores become
+// order-preserving 32-bit keys (-0 folded into +0, so equal scores stay
+// equal); each group's maximum is one warp max-reduction (redux.sync), and
+// every arg-max over the warp is a max-reduction of the lanes' best keys plus
+// a ballot: the lowest lane holding the maximum holds the lowest expert index.
+// The selections compare input scores only, so they are exact; the softmax
+// uses fp32 expf.  Scores must be finite.
 #pragma once
 
 #include "common.cuh"
@@ -31,86 +34,98 @@ struct RouteParams {
   float* topk_weights;
 };
 
-// (v, i) beats (w, j): higher score, then lower index
-__device__ __forceinline__ bool route_better(float v, int i, float w, int j) {
-  return v > w || (v == w && i < j);
+// Order-preserving key of a finite float: a > b  <=>  key(a) > key(b), and
+// key(-0) == key(+0).
+__device__ __forceinline__ int32_t route_key(float f) {
+  const int32_t i = __float_as_int(f + 0.0f);  // -0 + 0 = +0
+  return i >= 0 ? i : i ^ 0x7fffffff;
 }
 
-__device__ __forceinline__ void warp_argmax(float& v, int& i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float w = __shfl_xor_sync(0xffffffffu, v, o);
-    const int j = __shfl_xor_sync(0xffffffffu, i, o);
-    if (route_better(w, j, v, i)) {
-      v = w;
-      i = j;
-    }
-  }
-}
+constexpr int32_t kRouteNoKey = INT32_MIN;  // below every finite score's key
 
-// NQ = values per lane (E <= 32*NQ); the caller picks the smallest of
+// NQ = experts per lane (E <= 32*NQ); the caller picks the smallest of
 // 1, 2, 4, 8, 16, 32 that holds E.
 template <int NQ>
 __global__ void __launch_bounds__(kRouteThreads) route_group_limited_kernel(RouteParams p) {
   const int lane = threadIdx.x & (kWarp - 1);
   const int per = p.E / p.n_groups;
-  const float kNone = -__int_as_float(0x7f800000);  // -inf: below every finite score
+  const int e0 = lane * NQ;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp; t < p.T;
        t += static_cast<int64_t>(gridDim.x) * (kRouteThreads / kWarp)) {
     const float* s = p.scores + t * p.E;
     float v[NQ];
-    int gq[NQ];  // group of this lane's q-th expert, -1 past E
+    int32_t key[NQ];
+    int gq[NQ];  // group of expert e0+q, -1 past E
+    if (NQ % 4 == 0 && e0 + NQ <= p.E && (reinterpret_cast<uintptr_t>(s + e0) & 15) == 0) {
+#pragma unroll
+      for (int q = 0; q < NQ; q += 4) {
+        const float4 f = *reinterpret_cast<const float4*>(s + e0 + q);
+        v[q] = f.x;
+        v[q + 1] = f.y;
+        v[q + 2] = f.z;
+        v[q + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) v[q] = e0 + q < p.E ? s[e0 + q] : 0.0f;
+    }
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-      const int e = q * kWarp + lane;
+      const int e = e0 + q;
       const bool ok = e < p.E;
-      v[q] = ok ? s[e] : kNone;
+      key[q] = ok ? route_key(v[q]) : kRouteNoKey;
       gq[q] = ok ? e / per : -1;
     }
-    // group scores: lane g ends up holding the score of group g
-    float my_group = kNone;
+    // group scores: lane g keeps group g's key (one max-reduction per group)
+    int32_t my_gkey = kRouteNoKey;
     for (int g = 0; g < p.n_groups; ++g) {
-      float m = kNone;
+      int32_t m = kRouteNoKey;
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
-        if (gq[q] == g) m = fmaxf(m, v[q]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (lane == g) my_group = m;
+        if (gq[q] == g) m = max(m, key[q]);
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (lane == g) my_gkey = m;
     }
-    // the best groups, one arg-max per pick
+    // the chosen groups: per pick, the largest key, lowest group among equals
     uint32_t chosen = 0;
     for (int n = 0; n < p.topk_groups; ++n) {
       const bool cand = lane < p.n_groups && !((chosen >> lane) & 1u);
-      float gv = cand ? my_group : kNone;
-      int gi = cand ? lane : kWarp;
-      warp_argmax(gv, gi);
-      if (gi < kWarp) chosen |= 1u << gi;
+      const int32_t gk = cand ? my_gkey : kRouteNoKey;
+      const int32_t top = __reduce_max_sync(0xffffffffu, gk);
+      const uint32_t holders = __ballot_sync(0xffffffffu, cand && gk == top);
+      chosen |= 1u << (__ffs(holders) - 1);
     }
-    // candidates: this lane's experts in the chosen groups
-    uint32_t open = 0;  // bit q: expert q*32+lane is still a candidate
+    uint32_t open = 0;  // bit q: expert e0+q is still a candidate
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
       if (gq[q] >= 0 && ((chosen >> gq[q]) & 1u)) open |= 1u << q;
-    // the best experts, in order
+    // the best experts, in order: per round, each lane offers its best open
+    // expert (lowest index among equal keys), the warp takes the maximum key
+    // and, among lanes that hold it, the lowest lane
     float my_score = 0.0f;
     int my_expert = -1;
     for (int j = 0; j < p.k; ++j) {
-      float bv = kNone;
-      int bi = p.E;
+      int32_t bk = kRouteNoKey;
+      int bq = -1;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const int e = q * kWarp + lane;
-        if (((open >> q) & 1u) && route_better(v[q], e, bv, bi)) {
-          bv = v[q];
-          bi = e;
+      for (int q = 0; q < NQ; ++q)
+        if (((open >> q) & 1u) && key[q] > bk) {
+          bk = key[q];
+          bq = q;
         }
-      }
-      warp_argmax(bv, bi);
-      if (bi < p.E && (bi & (kWarp - 1)) == lane) open &= ~(1u << (bi / kWarp));
+      const int32_t top = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t holders = __ballot_sync(0xffffffffu, bq >= 0 && bk == top);
+      const int win = __ffs(holders) - 1;
+      float sv = 0.0f;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+        if (q == bq) sv = v[q];
+      const int wq = __shfl_sync(0xffffffffu, bq, win);
+      const float ws = __shfl_sync(0xffffffffu, sv, win);
+      if (lane == win) open &= ~(1u << wq);
       if (lane == j) {
-        my_score = bv;
-        my_expert = bi;
+        my_score = ws;
+        my_expert = win * NQ + wq;
       }
     }
     // softmax of the chosen scores (the first one is the largest)
