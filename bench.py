@@ -187,12 +187,12 @@ class ClockSampler:
 class Path:
     """Device buffers of one workload and one step through the C ABI."""
 
-    def __init__(self, w, d, dev, max_tokens_per_rank=0, route=False):
+    def __init__(self, w, d, dev, max_tokens_per_rank=0, route=False, num_sms=0):
         import numpy as np
         import torch
         import combine_ep_get_histogram_b200 as ep
         self.ep, self.w, self.dev = ep, w, dev
-        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8, 0, max_tokens_per_rank)
+        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8, num_sms, max_tokens_per_rank)
         P = ep.ep.receive_rows(self.shape)
 
         def bf16(a):
@@ -214,7 +214,10 @@ class Path:
         self.grad_w = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
         self.grad_x = torch.empty((w.T, w.H), dtype=torch.int16, device=dev)
 
-    def step(self, marks=None):
+    def step(self, marks=None, before_back=None, after_combine=None):
+        """One pass of the path.  before_back runs (on the host, at enqueue
+        time) between dispatch and combine, after_combine right after combine:
+        hooks for the end-to-end pipeline's stream waits and events."""
         ep, i = self.ep, self.inp
         n = 0
 
@@ -234,7 +237,11 @@ class Path:
         ep.ep_dispatch(self.shape, i["x"], i["topk_weights"], self.handle, self.recv_x, self.recv_scale,
                        self.recv_weight)
         rec()
+        if before_back is not None:
+            before_back()
         ep.ep_combine(self.shape, i["y"], i["topk_weights"], self.handle, self.out)
+        if after_combine is not None:
+            after_combine()
         rec()
         ep.ep_combine_backward(self.shape, i["g"], i["y"], i["topk_weights"], self.handle, self.grad_y,
                                self.grad_w)
@@ -329,37 +336,84 @@ def run_ours(args, rank, world, local):
     total_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
     ms_per_step = total_ms / args.steps
 
-    # end to end through the same C ABI: pinned host inputs in, results out, per step
+    # End to end through the same C ABI: every step copies its inputs from
+    # pinned host memory and reads its results back.  Two device buffer sets
+    # alternate, so step i+1's host-to-device copies (one stream) overlap step
+    # i's kernels (a second stream) and step i's device-to-host copies (a
+    # third stream; PCIe is full duplex).
     e2e = None
     if not args.no_e2e:
+        paths = [path, Path(w, d, dev, M, route=args.route)]
         pin = {n: t.pin_memory() for n, t in path.host.items()}
         outs = {"out": torch.empty_like(path.out, device="cpu").pin_memory(),
                 "grad_x": torch.empty_like(path.grad_x, device="cpu").pin_memory(),
                 "grad_w": torch.empty_like(path.grad_w, device="cpu").pin_memory()}
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
         d2h = sum(t.numel() * t.element_size() for t in outs.values())
+        back_names = ("g", "y")  # needed from combine on
+        front_names = tuple(n for n in pin if n not in back_names)
+        s_h2d, s_comp, s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
+        comp_done, d2h_done = [None, None], [None, None]
 
-        def e2e_step():
-            for n, t in pin.items():
-                path.inp[n].copy_(t, non_blocking=True)
-            path.step()
-            outs["out"].copy_(path.out, non_blocking=True)
-            outs["grad_x"].copy_(path.grad_x, non_blocking=True)
-            outs["grad_w"].copy_(path.grad_w, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            p = paths[b]
+            ev_front, ev_back, ev_out = (torch.cuda.Event() for _ in range(3))
+            with torch.cuda.stream(s_h2d):
+                if comp_done[b] is not None:  # step i-2 has finished reading these inputs
+                    s_h2d.wait_event(comp_done[b])
+                for n in front_names:
+                    p.inp[n].copy_(pin[n], non_blocking=True)
+                ev_front.record(s_h2d)
+                for n in back_names:
+                    p.inp[n].copy_(pin[n], non_blocking=True)
+                ev_back.record(s_h2d)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(ev_front)
+                if d2h_done[b] is not None:  # step i-2's results have left these outputs
+                    s_comp.wait_event(d2h_done[b])
+                p.step(before_back=lambda: s_comp.wait_event(ev_back), after_combine=lambda: ev_out.record(s_comp))
+                comp_done[b] = torch.cuda.Event()
+                comp_done[b].record(s_comp)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev_out)
+                outs["out"].copy_(p.out, non_blocking=True)
+                s_d2h.wait_event(comp_done[b])
+                outs["grad_x"].copy_(p.grad_x, non_blocking=True)
+                outs["grad_w"].copy_(p.grad_w, non_blocking=True)
+                d2h_done[b] = torch.cuda.Event()
+                d2h_done[b].record(s_d2h)
 
-        for _ in range(max(1, min(args.warmup, 3))):
-            e2e_step()
+        def join(cur):
+            for st in (s_h2d, s_comp, s_d2h):
+                ev = torch.cuda.Event()
+                ev.record(st)
+                cur.wait_event(ev)
+
+        cur = torch.cuda.current_stream()
+        for i in range(max(2, min(args.warmup, 4))):
+            e2e_step(i)
+        join(cur)
         barrier()
-        n_e2e = max(1, min(args.steps, 10))
+        n_e2e = max(2, min(args.steps, 10))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record()
+        e0.record(cur)
+        for st in (s_h2d, s_comp, s_d2h):
+            st.wait_event(e0)
+        for i in range(n_e2e):
+            e2e_step(i)
+        join(cur)
+        e1.record(cur)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"value": round(job_gbs(step_bytes, n_e2e, world, e_ms), 2), "unit": "GB/s",
-               "ms_per_step": round(e_ms / n_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "ms_per_step": round(e_ms / n_e2e, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": n_e2e,
+               "pipelining": "two device buffer sets; step i+1's host-to-device copies overlap step i's "
+                             "kernels and its device-to-host copies (three streams)"}
+        del paths[1]
+
+    overlap = measure_overlap(args, w, d, dev, M, ms_per_step) if args.overlap_sms else None
 
     if rank != 0:
         return None
@@ -409,7 +463,75 @@ def run_ours(args, rank, world, local):
         "timing": "CUDA graph replay of the step" if not args.no_graph else "eager launches",
         "e2e": e2e,
     }
+    if overlap is not None:
+        line["overlap"] = overlap
     return line
+
+
+def measure_overlap(args, w, d, dev, M, step_ms):
+    """The path on a side stream with an SM budget of N beside a
+    compute-bound cuBLAS GEMM on the launching stream that leaves N SMs free
+    (torch's matmul SM carve-out), against the best serial schedule: the GEMM
+    on all SMs, then the path on all SMs.  The GEMM repeats are sized to
+    about one full-GPU step of the path."""
+    import torch
+    budget = Path(w, d, dev, M, route=args.route, num_sms=args.overlap_sms)
+    full = Path(w, d, dev, M, route=args.route)
+    n = 8192
+    gen = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randn((n, n), device=dev, dtype=torch.bfloat16, generator=gen)
+    b = torch.randn((n, n), device=dev, dtype=torch.bfloat16, generator=gen)
+    c = torch.empty((n, n), device=dev, dtype=torch.bfloat16)
+    cur = torch.cuda.current_stream()
+    side = torch.cuda.Stream(dev)
+
+    def timed(fn, iters=5):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        for _ in range(iters):
+            fn()
+        e1.record(cur)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    one = timed(lambda: torch.matmul(a, b, out=c))
+    reps = max(1, round(step_ms / one))
+
+    def gemms(carveout=None):
+        torch._C._set_sm_carveout_experimental(carveout)
+        try:
+            for _ in range(reps):
+                torch.matmul(a, b, out=c)
+        finally:
+            torch._C._set_sm_carveout_experimental(None)
+
+    def serial():
+        gemms()
+        full.step()
+
+    def overlapped():
+        ev = torch.cuda.Event()
+        ev.record(cur)
+        side.wait_event(ev)
+        with torch.cuda.stream(side):
+            budget.step()
+        gemms(args.overlap_sms)
+        done = torch.cuda.Event()
+        done.record(side)
+        cur.wait_event(done)
+
+    t_gemm, t_gemm_carved = timed(gemms), timed(lambda: gemms(args.overlap_sms))
+    t_path, t_path_budget = timed(full.step), timed(budget.step)
+    t_serial, t_over = timed(serial), timed(overlapped)
+    return {"num_sms": args.overlap_sms, "gemm": f"torch.matmul bf16 {n}x{n}x{n} x {reps}",
+            "gemm_ms_all_sms": round(t_gemm, 3), "gemm_ms_carved": round(t_gemm_carved, 3),
+            "path_ms_all_sms": round(t_path, 3), "path_ms_at_budget": round(t_path_budget, 3),
+            "serial_ms": round(t_serial, 3), "overlapped_ms": round(t_over, 3),
+            "saved_frac": round(1.0 - t_over / t_serial, 3),
+            "timing": "CUDA events on the launching stream, eager launches, mean of 5"}
 
 
 def workload(args):
@@ -488,7 +610,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each call eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-tokens-per-rank", type=int, default=512)
+    ap.add_argument("--overlap-sms", type=int, default=0,
+                    help="also time the path with this SM budget on a side stream beside a bf16 GEMM")
+    ap.add_argument("--cpu-tokens-per-rank", type=int, default=1536)
     ap.add_argument("--ref-tokens-per-rank", type=int, default=64)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -93,8 +93,18 @@ typedef enum {
 typedef struct {
   int32_t T, H, k, E, R;
   int32_t use_fp8; /* 1: dispatch writes E4M3 codes + fp32 scales; 0: bf16 rows */
-  int32_t num_sms; /* SMs a call may fill: 0 = all.  Caps each grid at
-                      num_sms x (resident CTAs per SM). */
+  int32_t num_sms; /* SM budget of the data-movement kernels (dispatch,
+                      combine, both backward passes) and the router: 0 or a
+                      value >= the device's SM count = all SMs; else each of
+                      their grids is capped at num_sms x (CTAs of that kernel
+                      resident per SM), so the caller's own kernels keep the
+                      rest (blog.hotdry.top, section 二, SM 资源控制).  The
+                      hardware places a grid's CTAs on distinct SMs before it
+                      stacks them, so the CTAs land on num_sms SMs only when
+                      the stream belongs to an SM partition of that size (a
+                      CUDA green context).  The layout kernels (tens of
+                      microseconds) are not capped.  Results do not depend on
+                      the budget. */
   int32_t max_tokens_per_rank; /* 0: dense receive layout (below).  M > 0:
                       the padded low-latency layout: E*R*M receive rows, one
                       block of M rows per (expert e, source rank r) at row

@@ -9,61 +9,10 @@ import numpy as np
 import pytest
 import torch
 
-import combine_ep_get_histogram_b200 as ep
 from combine_ep_get_histogram_b200 import workloads as wl
-from gpu_util import to_dev
+from gpu_util import StepBuffers as Step
 
 pytestmark = pytest.mark.gpu
-
-
-class Step:
-    def __init__(self, w, device, max_tokens_per_rank=0):
-        self.w = w
-        self.shape = ep.make_shape(w.T, w.H, w.k, w.E, w.R, w.use_fp8, 0, max_tokens_per_rank)
-        P = ep.ep.receive_rows(self.shape)
-        self.h = ep.Handle(self.shape, device)
-        self.ws = ep.workspace(self.shape, device)
-        self.idx = torch.empty((w.T, w.k), dtype=torch.int64, device=device)
-        self.wts = torch.empty((w.T, w.k), dtype=torch.float32, device=device)
-        self.x = torch.empty((w.T, w.H), dtype=torch.int16, device=device)
-        self.y = torch.empty((P, w.H), dtype=torch.int16, device=device)
-        self.g = torch.empty((w.T, w.H), dtype=torch.int16, device=device)
-        self.rx = torch.empty((P, w.H), dtype=torch.uint8 if w.use_fp8 else torch.int16, device=device)
-        self.rs = torch.empty((P, w.G), dtype=torch.float32, device=device) if w.use_fp8 else None
-        self.rw = torch.empty(P, dtype=torch.float32, device=device)
-        self.out = torch.empty((w.T, w.H), dtype=torch.int16, device=device)
-        self.gy = torch.empty((P, w.H), dtype=torch.int16, device=device)
-        self.gw = torch.empty((w.T, w.k), dtype=torch.float32, device=device)
-        self.gx = torch.empty((w.T, w.H), dtype=torch.int16, device=device)
-
-    def load(self, d):
-        self.idx.copy_(torch.from_numpy(d["topk_idx"]))
-        self.wts.copy_(torch.from_numpy(d["topk_weights"]))
-        for n in ("x", "y", "g"):
-            getattr(self, n).copy_(to_dev(d[n], "cpu"))
-
-    def run(self):
-        ep.ep_get_dispatch_layout(self.shape, self.idx, self.h, self.ws)
-        ep.ep_dispatch(self.shape, self.x, self.wts, self.h, self.rx, self.rs, self.rw)
-        ep.ep_combine(self.shape, self.y, self.wts, self.h, self.out)
-        ep.ep_combine_backward(self.shape, self.g, self.y, self.wts, self.h, self.gy, self.gw)
-        ep.ep_dispatch_backward(self.shape, self.gy, self.h, self.gx)
-
-    def outputs(self):
-        """Handle arrays, and the receive rows that hold a pair (padded
-        layouts leave the other rows unwritten)."""
-        torch.cuda.synchronize()
-        if self.shape.max_tokens_per_rank:
-            rows = torch.nonzero(self.h.src_of_slot >= 0).squeeze(1)
-        else:
-            rows = torch.arange(int(self.h.expert_offset[-1].item()), device=self.rx.device)
-        res = [self.h.tensors[f].clone() for f in ("slot_of_pair", "src_of_slot", "expert_offset",
-                                                    "num_tokens_per_rank", "is_token_in_rank")]
-        res += [self.rx[rows].clone(), self.rw[rows].clone(), self.out.clone(), self.gy[rows].clone(),
-                self.gw.clone(), self.gx.clone()]
-        if self.rs is not None:
-            res.append(self.rs[rows].clone())
-        return res
 
 
 @pytest.mark.parametrize("name,padded", [("decode", False), ("tiny", False), ("tiny", True)])
