@@ -35,7 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-METRIC = "dispatch/combine µs/call & effective GB/s vs B200 roofline, 1 GPU"
+METRIC = "dispatch/combine µs/call & effective HBM GB/s vs B200 roofline, 1 GPU"
 CALLS = ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward")
 ROUTE_CALLS = ("route",) + CALLS
 FALLBACK_HBM_GBS = 6650.0
@@ -258,6 +258,21 @@ def launches_per_step(w) -> int:
     return (1 if small else 3) + 4
 
 
+def bench_config(w, args, world: int) -> dict:
+    """The JSON line's config: the workload by name and sizes (both arms)."""
+    return {"workload": f"{w.name}: T={w.T} ({w.R} virtual ranks x {w.T // w.R} tokens), H={w.H}, "
+                        f"E={w.E}, k={w.k}, top-{w.topk_groups} of {w.n_groups} groups, "
+                        f"{'FP8' if w.use_fp8 else 'BF16'} dispatch + BF16 combine + both backward passes",
+            "T": w.T, "H": w.H, "k": w.k, "E": w.E, "R": w.R, "use_fp8": w.use_fp8,
+            "storage": ("e4m3 codes + f32 scales dispatched, bf16 expert rows, outputs and gradients"
+                        if w.use_fp8 else "bf16 rows, outputs and gradients"),
+            "step_bytes": sum(call_bytes(w)[c] for c in step_calls(args)), "l2": "inputs larger than L2 (no flush)",
+            "receive_layout": (f"padded [E][R][{args.max_tokens_per_rank}]" if args.max_tokens_per_rank
+                               else "dense [T*k]"),
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, virtual ranks",
+            "router_in_step": bool(args.route)}
+
+
 def run_ours(args, rank, world, local):
     import numpy as np
     import torch
@@ -268,7 +283,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.set_device(dev)
     w = workload(args)
     M = args.max_tokens_per_rank
-    calls = ROUTE_CALLS if args.route else CALLS
+    calls = step_calls(args)
     d = wl.make_inputs(w, parts=("routing", "x", "g") + (() if M else ("y",)) + (("scores",) if args.route else ()))
     if M:  # expert outputs fill the padded receive rows
         d["y"] = wl.normal_bf16(w.E * w.R * M, w.H, w.seed, 2)
@@ -442,16 +457,9 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8-e4m3 dispatch / bf16 combine, fp32 math" if w.use_fp8 else "bf16, fp32 math",
+        "dtype": "f32",
         "data": "synthetic (seeded group-limited routing, N(0,1) activations)",
-        "config": {"workload": f"{w.name}: T={w.T} ({w.R} virtual ranks x {w.T // w.R} tokens), H={w.H}, "
-                               f"E={w.E}, k={w.k}, top-{w.topk_groups} of {w.n_groups} groups, "
-                               f"{'FP8' if w.use_fp8 else 'BF16'} dispatch + BF16 combine + both backward passes",
-                   "T": w.T, "H": w.H, "k": w.k, "E": w.E, "R": w.R, "use_fp8": w.use_fp8,
-                   "step_bytes": step_bytes, "l2": "inputs larger than L2 (no flush)",
-                   "receive_layout": (f"padded [E][R][{args.max_tokens_per_rank}]" if args.max_tokens_per_rank
-                                      else "dense [T*k]"),
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, virtual ranks"},
+        "config": bench_config(w, args, world),
         "per_call": per_call,
         "roofline": {"kernel": kernel_of[dominant], "call": dominant, "bound": "hbm", "achieved": ach,
                      "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 3),
@@ -539,56 +547,80 @@ def workload(args):
     w = wl.CONFIGS[args.workload]
     if args.tokens_per_rank:
         w = w.with_(T=w.R * args.tokens_per_rank)
+    if args.dispatch_dtype != "default":
+        w = w.with_(use_fp8=args.dispatch_dtype == "fp8")
     return w
 
 
 # -------------------------------------------------------- CPU oracle arm
 
-def oracle_pass(w, d):
+def step_calls(args) -> tuple:
+    return ROUTE_CALLS if args.route else CALLS
+
+
+def oracle_pass(w, d, route: bool, M: int):
+    """One step of the path on the oracle: routing (if timed), the dense or
+    padded layout, dispatch, combine and both backward passes."""
     import oracle
-    lay = oracle.layout(d["topk_idx"], w.E, w.R)
+    idx, wts = d["topk_idx"], d["topk_weights"]
+    if route:
+        idx, wts = oracle.route_group_limited(d["scores"], w.k, w.n_groups, w.topk_groups)
+    if M:
+        lay, rows = oracle.layout_padded(idx, w.E, w.R, M), w.E * w.R * M
+    else:
+        lay, rows = oracle.layout(idx, w.E, w.R), w.T * w.k
     slots = lay["slot_of_pair"]
-    oracle.dispatch(d["x"], d["topk_weights"], slots, w.use_fp8)
-    oracle.combine(d["y"], d["topk_weights"], slots)
-    gy, _ = oracle.combine_backward(d["g"], d["y"], d["topk_weights"], slots)
+    oracle.dispatch(d["x"], wts, slots, w.use_fp8, P=rows)
+    oracle.combine(d["y"], wts, slots)
+    gy, _ = oracle.combine_backward(d["g"], d["y"], wts, slots, P=rows)
     oracle.dispatch_backward(gy, slots, w.T, w.k)
 
 
-def cpu_sample(workload: str, tokens_per_rank: int):
+def cpu_sample(args, tokens_per_rank: int):
+    """The bench's workload (dispatch dtype override, routing and receive
+    layout included) cut to tokens_per_rank tokens per virtual rank.  A
+    padded layout gets tokens_per_rank rows per (expert, source rank) block."""
     from combine_ep_get_histogram_b200 import workloads as wl
-    w = wl.CONFIGS[workload]
+    w = workload(args)
     ws = w.with_(T=w.R * tokens_per_rank)
-    d = wl.make_inputs(ws, parts=("routing", "x", "y", "g"))
+    M = tokens_per_rank if args.max_tokens_per_rank else 0
+    d = wl.make_inputs(ws, parts=("routing", "x", "g") + (() if M else ("y",)) +
+                       (("scores",) if args.route else ()))
+    if M:
+        d["y"] = wl.normal_bf16(ws.E * ws.R * M, ws.H, ws.seed, 2)
     desc = (f"{w.name} shape (H={w.H}, E={w.E}, k={w.k}, R={w.R}) with T={ws.T} "
-            f"({tokens_per_rank} tokens per rank) instead of {w.T}; one full pass of the five calls")
-    return ws, d, desc
+            f"({tokens_per_rank} tokens per rank) instead of {w.T}"
+            + (f", padded blocks of {M} rows" if M else "")
+            + f"; one full pass of the step ({', '.join(step_calls(args))})")
+    return ws, d, desc, M
 
 
 def run_cpu_baseline(args) -> dict:
-    ws, d, desc = cpu_sample(args.workload, args.cpu_tokens_per_rank)
+    ws, d, desc, M = cpu_sample(args, args.cpu_tokens_per_rank)
     t = time.perf_counter()
-    oracle_pass(ws, d)
+    oracle_pass(ws, d, args.route, M)
     dt = time.perf_counter() - t
-    gbs = sum(call_bytes(ws).values()) / dt / 1e9
+    gbs = sum(call_bytes(ws)[c] for c in step_calls(args)) / dt / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
             "seconds": round(dt, 2)}
 
 
 def run_reference(args) -> dict:
-    ws, d, desc = cpu_sample(args.workload, args.ref_tokens_per_rank)
+    ws, d, desc, M = cpu_sample(args, args.ref_tokens_per_rank)
     for _ in range(args.warmup):
-        oracle_pass(ws, d)
+        oracle_pass(ws, d, args.route, M)
     t = time.perf_counter()
     for _ in range(args.steps):
-        oracle_pass(ws, d)
+        oracle_pass(ws, d, args.route, M)
     dt = (time.perf_counter() - t) / args.steps
-    gbs = sum(call_bytes(ws).values()) / dt / 1e9
+    gbs = sum(call_bytes(ws)[c] for c in step_calls(args)) / dt / 1e9
     return {
-        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 0,
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "device": "host cores (rank 0 only)",
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8-e4m3 dispatch / bf16 combine, fp32 math" if ws.use_fp8 else "bf16, fp32 math",
-        "data": "synthetic (seeded)", "config": {"workload": desc},
+        "dtype": "f32",
+        "data": "synthetic (seeded)", "config": bench_config(workload(args), args, 1),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -605,6 +637,8 @@ def main():
                     help="start each step with group-limited routing of [T,E] scores (the step before the path)")
     ap.add_argument("--max-tokens-per-rank", type=int, default=0,
                     help="padded low-latency receive layout with this many rows per (expert, source rank)")
+    ap.add_argument("--dispatch-dtype", choices=("default", "bf16", "fp8"), default="default",
+                    help="override the workload's dispatch payload (the skewed workload is timed with both)")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="resize the workload to R x this many tokens (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")

@@ -69,6 +69,7 @@ def _run_reference(rank: int):
 
 
 def test_reference_arm_prints_on_rank_zero_only():
+    import bench
     r1 = _run_reference(1)
     assert r1.returncode == 0 and r1.stdout.strip() == ""
     r0 = _run_reference(0)
@@ -76,3 +77,20 @@ def test_reference_arm_prints_on_rank_zero_only():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["n_gpus"] == 2 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["higher_is_better"] is True and line["unit"] == line["e2e"]["unit"] == "GB/s"
+    # the same workload and config as the GPU arm's line
+    assert line["config"]["workload"].startswith("prefill: T=32768") and line["config"]["H"] == 7168
+    nb = bench.call_bytes(bench.workload(_default_args()))
+    assert line["config"]["step_bytes"] == sum(nb[c] for c in bench.CALLS)
+    for key in ("value", "unit", "cores", "kind", "sample"):
+        assert key in line["cpu_baseline"], key
+
+
+def _default_args():
+    import argparse
+    return argparse.Namespace(workload="prefill", tokens_per_rank=0, dispatch_dtype="default", route=False,
+                              max_tokens_per_rank=0)
