@@ -42,7 +42,8 @@ struct DeviceInfo {
   int occ_disp_bf16 = 0, occ_disp_fp8 = 0, occ_comb = 0, occ_dbwd = 0;
   int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
   int occ_cbwd = 0;
-  int occ_route[6] = {};  // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
+  int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
+  int occ_route_aligned[6] = {};  // route_aligned_kernel<1, 2, 4, 8, 16, 32>
 };
 
 constexpr int kMaxDevices = 64;
@@ -85,7 +86,16 @@ int device_info(const DeviceInfo** out) {
                                   reinterpret_cast<const void*>(route_group_limited_kernel<8>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<16>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<32>)};
-      for (int i = 0; i < 6; ++i) d.occ_route[i] = occupancy(route_fns[i], kRouteThreads, 0);
+      const void* aligned_fns[6] = {reinterpret_cast<const void*>(route_aligned_kernel<1>),
+                                    reinterpret_cast<const void*>(route_aligned_kernel<2>),
+                                    reinterpret_cast<const void*>(route_aligned_kernel<4>),
+                                    reinterpret_cast<const void*>(route_aligned_kernel<8>),
+                                    reinterpret_cast<const void*>(route_aligned_kernel<16>),
+                                    reinterpret_cast<const void*>(route_aligned_kernel<32>)};
+      for (int i = 0; i < 6; ++i) {
+        d.occ_route[i] = occupancy(route_fns[i], kRouteThreads, 0);
+        d.occ_route_aligned[i] = occupancy(aligned_fns[i], kRouteThreads, 0);
+      }
       cudaGetLastError();
     }
     g_dev[dev] = d;
@@ -385,13 +395,30 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
   if ((st = device_info(&d)) != EP_OK) return st;
   if (T == 0) return EP_OK;
   RouteParams p{scores, shape->T, shape->E, shape->k, n_groups, topk_groups, topk_idx, topk_weights};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   constexpr int warps = kRouteThreads / kWarp;
   const int nq = static_cast<int>(ceil_div(shape->E, kWarp));
   const int variant = nq <= 1 ? 0 : nq <= 2 ? 1 : nq <= 4 ? 2 : nq <= 8 ? 3 : nq <= 16 ? 4 : 5;
-  const int64_t cap = grid_cap(*d, shape, d->occ_route[variant]);
+  // groups on lane boundaries: a lane's experts share one group and a group
+  // spans a power-of-two number of lanes
+  const int per_lane = 1 << variant, per_group = shape->E / n_groups;
+  const int lanes_per_group = per_group / per_lane;
+  const bool on_lanes = shape->E % per_lane == 0 && per_group % per_lane == 0 &&
+                        (lanes_per_group & (lanes_per_group - 1)) == 0;
+  const int64_t cap = grid_cap(*d, shape, on_lanes ? d->occ_route_aligned[variant] : d->occ_route[variant]);
   const int64_t need = ceil_div(T, warps);
   const int grid = static_cast<int>(need < cap ? need : cap);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (on_lanes) {
+    switch (variant) {
+      case 0: route_aligned_kernel<1><<<grid, kRouteThreads, 0, s>>>(p); break;
+      case 1: route_aligned_kernel<2><<<grid, kRouteThreads, 0, s>>>(p); break;
+      case 2: route_aligned_kernel<4><<<grid, kRouteThreads, 0, s>>>(p); break;
+      case 3: route_aligned_kernel<8><<<grid, kRouteThreads, 0, s>>>(p); break;
+      case 4: route_aligned_kernel<16><<<grid, kRouteThreads, 0, s>>>(p); break;
+      default: route_aligned_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
+    }
+    return cuda_status(cudaGetLastError());
+  }
   switch (variant) {
     case 0: route_group_limited_kernel<1><<<grid, kRouteThreads, 0, s>>>(p); break;
     case 1: route_group_limited_kernel<2><<<grid, kRouteThreads, 0, s>>>(p); break;

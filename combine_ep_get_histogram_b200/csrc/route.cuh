@@ -12,11 +12,21 @@
 // One warp per token.  Lane l holds the scores of the contiguous experts
 // [l*NQ, (l+1)*NQ), so lane order is expert order.  Scores become
 // order-preserving 32-bit keys (-0 folded into +0, so equal scores stay
-// equal); each group's maximum is one warp max-reduction (redux.sync), and
-// every arg-max over the warp is a max-reduction of the lanes' best keys plus
-// a ballot: the lowest lane holding the maximum holds the lowest expert index.
-// The selections compare input scores only, so they are exact; the softmax
-// uses fp32 expf.  Scores must be finite.
+// equal).  Every arg-max over the warp is a max-reduction (redux.sync) of the
+// lanes' best keys plus a ballot: the lowest lane holding the maximum holds
+// the lowest expert index.  The selections compare input scores only, so
+// they are exact; the softmax uses fp32 expf.  Scores must be finite.
+//
+// Two kernels.  route_aligned_kernel serves shapes whose groups fall on lane
+// boundaries (E and the group size multiples of NQ, and a power-of-two
+// number of lanes per group; 256 experts in 8 groups is one): a group's
+// maximum is the lanes' maxima combined by xor shuffles inside the group's
+// lane segment, a group's rank is counted from one shuffle per group, each
+// lane sorts its candidates once (a bitonic network over 64-bit (key,
+// expert) composites), and a pick takes the largest first key over the
+// warp, the winning lane dropping its first entry.
+// route_group_limited_kernel serves every other shape: one warp
+// max-reduction per group over per-expert group ids.
 #pragma once
 
 #include "common.cuh"
@@ -129,6 +139,128 @@ __global__ void __launch_bounds__(kRouteThreads) route_group_limited_kernel(Rout
       }
     }
     // softmax of the chosen scores (the first one is the largest)
+    const float top = __shfl_sync(0xffffffffu, my_score, 0);
+    const float ex = lane < p.k ? expf(my_score - top) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < p.k) {
+      p.topk_idx[t * p.k + lane] = my_expert;
+      p.topk_weights[t * p.k + lane] = __fdiv_rn(ex, sum);
+    }
+  }
+}
+
+// Order of a candidate within a lane: larger composite = earlier (larger
+// key, then lower local index q).  0 is below every candidate.
+__device__ __forceinline__ uint64_t route_composite(int32_t key, int q) {
+  return (static_cast<uint64_t>(static_cast<uint32_t>(key) ^ 0x80000000u) << 32) |
+         static_cast<uint64_t>(0xFFFFFFFFu - static_cast<uint32_t>(q));
+}
+
+// The score whose key is `key` (-0 comes back as +0, which changes no
+// difference taken from it).
+__device__ __forceinline__ float route_score(int32_t key) {
+  return __int_as_float(key >= 0 ? key : key ^ 0x7fffffff);
+}
+
+__device__ __forceinline__ void route_cas(uint64_t& a, uint64_t& b) {  // a >= b afterwards
+  const bool swap = b > a;
+  const uint64_t hi = swap ? b : a;
+  b = swap ? a : b;
+  a = hi;
+}
+
+// Descending bitonic sort of N (a power of two) composites.
+template <int N>
+__device__ __forceinline__ void route_sort_desc(uint64_t (&a)[N]) {
+#pragma unroll
+  for (int k = 2; k <= N; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          if ((i & k) == 0)
+            route_cas(a[i], a[l]);
+          else
+            route_cas(a[l], a[i]);
+        }
+      }
+}
+
+// Groups on lane boundaries: E % NQ == 0, (E / n_groups) % NQ == 0 and
+// lpg = E / n_groups / NQ a power of two, so group g is lanes
+// [g*lpg, (g+1)*lpg) and lanes from E/NQ on hold no expert.  Each lane sorts
+// its candidates once; a pick is a max-reduction of the lanes' first keys, a
+// ballot (the lowest lane among equal keys holds the lowest expert), and the
+// winning lane drops its first entry.
+template <int NQ>
+__global__ void __launch_bounds__(kRouteThreads) route_aligned_kernel(RouteParams p) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int lpg = p.E / p.n_groups / NQ;
+  const int e0 = lane * NQ;
+  const bool has = e0 < p.E;
+  const int my_g = lane / lpg;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp; t < p.T;
+       t += static_cast<int64_t>(gridDim.x) * (kRouteThreads / kWarp)) {
+    const float* s = p.scores + t * p.E;
+    float v[NQ];
+    if (NQ % 4 == 0 && has && (reinterpret_cast<uintptr_t>(s + e0) & 15) == 0) {
+#pragma unroll
+      for (int q = 0; q < NQ; q += 4) {
+        const float4 f = *reinterpret_cast<const float4*>(s + e0 + q);
+        v[q] = f.x;
+        v[q + 1] = f.y;
+        v[q + 2] = f.z;
+        v[q + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) v[q] = has ? s[e0 + q] : 0.0f;
+    }
+    int32_t gk = kRouteNoKey;
+    uint64_t c[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int32_t key = has ? route_key(v[q]) : kRouteNoKey;
+      gk = max(gk, key);
+      c[q] = has ? route_composite(key, q) : 0;
+    }
+    // group maximum over the group's lane segment
+    for (int o = 1; o < lpg; o <<= 1) gk = max(gk, __shfl_xor_sync(0xffffffffu, gk, o));
+    // rank of this lane's group: groups with a larger maximum, or an equal
+    // one and a lower index
+    int rank = 0;
+    for (int g = 0; g < p.n_groups; ++g) {
+      const int32_t other = __shfl_sync(0xffffffffu, gk, g * lpg);
+      rank += (other > gk || (other == gk && g < my_g)) ? 1 : 0;
+    }
+    if (!(has && rank < p.topk_groups)) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) c[q] = 0;
+    }
+    route_sort_desc<NQ>(c);
+    int32_t my_key = 0;
+    int my_expert = -1;
+    for (int j = 0; j < p.k; ++j) {
+      const uint32_t head = static_cast<uint32_t>(c[0] >> 32);
+      const uint32_t top = __reduce_max_sync(0xffffffffu, head);
+      const int win = __ffs(__ballot_sync(0xffffffffu, head == top)) - 1;
+      const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(c[0]), win);
+      if (lane == j) {
+        my_key = static_cast<int32_t>(top ^ 0x80000000u);
+        my_expert = win * NQ + static_cast<int>(0xFFFFFFFFu - lo);
+      }
+      if (lane == win) {
+#pragma unroll
+        for (int q = 0; q + 1 < NQ; ++q) c[q] = c[q + 1];
+        c[NQ - 1] = 0;
+      }
+    }
+    // softmax of the chosen scores (the first one is the largest)
+    const float my_score = lane < p.k ? route_score(my_key) : 0.0f;
     const float top = __shfl_sync(0xffffffffu, my_score, 0);
     const float ex = lane < p.k ? expf(my_score - top) : 0.0f;
     float sum = ex;

@@ -1,4 +1,6 @@
-"""Group-limited top-k routing on the GPU against the oracle.
+"""Group-limited top-k routing on the GPU against the oracle, through both
+kernels: groups on lane boundaries (the aligned kernel) and off them (the
+general kernel).
 
 The selections compare input scores only, so topk_idx must match exactly
 (ties included: many scores are quantised to force them); the weights are
@@ -34,12 +36,22 @@ def route_gpu(device, s, k, ng, tg, R=1):
 
 
 @pytest.mark.parametrize("T,E,k,ng,tg", [
+    # groups on lane boundaries
     (1024, 256, 8, 8, 4),      # decode shape: top-4 of 8 groups, top-8 experts
     (32768, 256, 8, 8, 4),     # prefill shape
-    (512, 1024, 32, 32, 16),   # E and k at their maxima, 32 groups
     (300, 48, 6, 3, 2),        # E not a multiple of 32, 16 experts per group
     (200, 64, 5, 1, 1),        # one group: plain top-k
+    (77, 256, 3, 32, 1),       # one group of 8 chosen out of 32
+    (512, 1024, 32, 32, 16),   # E and k at their maxima, 32 groups
     (100, 16, 16, 4, 4),       # every expert chosen
+    # groups off lane boundaries: 12 experts per group over lanes of 4, 40
+    # over lanes of 8, E not a multiple of the experts per lane
+    (257, 96, 8, 8, 4),
+    (150, 160, 8, 4, 2),
+    (200, 33, 4, 3, 2),
+    (257, 96, 12, 8, 4),
+    (150, 160, 10, 4, 2),
+    (64, 300, 9, 3, 2),
 ])
 def test_route_matches_oracle(cuda_device, T, E, k, ng, tg):
     s = scores_for(T, E, seed=T + E + k)
