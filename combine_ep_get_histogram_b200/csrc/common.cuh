@@ -13,7 +13,14 @@ constexpr int kMaxR = 256;
 constexpr int kGroup = 128;                   // channels per FP8 scale
 constexpr int kLaneElems = 16;                // channels a lane moves per chunk
 constexpr int kChunk = kWarp * kLaneElems;    // 512 channels per warp chunk
-constexpr int kLanesPerGroup = kGroup / kLaneElems;  // 8
+// A lane's 16 channels of a chunk are two 8-channel pieces (16 bytes of
+// bf16 each) half a chunk apart: lane l holds [c*512 + 8l, +8) and
+// [c*512 + 256 + 8l, +8), so each 16-byte load or store of the warp covers
+// 512 contiguous bytes (16 sectors per request), and an FP8 scale group (128
+// channels) is one half-warp's pieces.
+constexpr int kPieceElems = 8;
+constexpr int kHalfChunk = kChunk / 2;        // 256: offset of a lane's second piece
+constexpr int kLanesPerGroup = kGroup / kPieceElems;  // 16
 constexpr int kTilePairs = 1024;              // layout tile: pairs per CTA
 constexpr int kTileFlagBytes = 32768;         // layout tile: tokens x ranks flag bytes
 constexpr int kLayoutThreads = 256;
@@ -89,6 +96,15 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* f) {
 __device__ __forceinline__ uint4 pack8_bf16(const float* f) {
   return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+}
+
+// First channel of a lane's first piece in chunk c (the second is kHalfChunk further).
+__device__ __forceinline__ int piece_channel(int c, int lane) { return c * kChunk + lane * kPieceElems; }
+
+// Eight fp32 values -> eight E4M3 codes, channel order in memory order.
+__device__ __forceinline__ uint2 pack8_e4m3(const float* f) {
+  return make_uint2(pack_e4m3x2(f[0], f[1]) | (pack_e4m3x2(f[2], f[3]) << 16),
+                    pack_e4m3x2(f[4], f[5]) | (pack_e4m3x2(f[6], f[7]) << 16));
 }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {

@@ -39,9 +39,10 @@ struct DeviceInfo {
   int sms = 0;
   bool supported = false;
   int occ_count = 0, occ_scan = 0, occ_assign = 0;
-  int occ_disp_bf16 = 0, occ_disp_fp8 = 0, occ_comb = 0, occ_dbwd = 0;
+  int occ_disp_bf16 = 0, occ_disp_fp8 = 0;
+  int occ_comb[2] = {}, occ_dbwd[2] = {};  // [ragged]
   int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
-  int occ_cbwd = 0;
+  int occ_cbwd[2] = {};  // [ragged]
   int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
   int occ_route_aligned[6] = {};  // route_aligned_kernel<1, 2, 4, 8, 16, 32>
 };
@@ -77,9 +78,12 @@ int device_info(const DeviceInfo** out) {
                               (kMaxE + kMaxR) * 4 + kTileFlagBytes);
       d.occ_disp_bf16 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<false>), kMoveThreads, 0);
       d.occ_disp_fp8 = occupancy(reinterpret_cast<const void*>(dispatch_kernel<true>), kMoveThreads, 0);
-      d.occ_comb = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<true>), kMoveThreads, 0);
-      d.occ_dbwd = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false>), kMoveThreads, 0);
-      d.occ_cbwd = occupancy(reinterpret_cast<const void*>(combine_backward_kernel), kMoveThreads, 0);
+      d.occ_comb[0] = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<true, false>), kMoveThreads, 0);
+      d.occ_comb[1] = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<true, true>), kMoveThreads, 0);
+      d.occ_dbwd[0] = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false, false>), kMoveThreads, 0);
+      d.occ_dbwd[1] = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false, true>), kMoveThreads, 0);
+      d.occ_cbwd[0] = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<false>), kMoveThreads, 0);
+      d.occ_cbwd[1] = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<true>), kMoveThreads, 0);
       const void* route_fns[6] = {reinterpret_cast<const void*>(route_group_limited_kernel<1>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<2>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<4>),
@@ -338,8 +342,14 @@ int ep_combine(const ep_shape_t* shape, const void* y, const float* topk_weights
   if (T == 0) return EP_OK;
   const MoveParams p = move_params(shape, handle, topk_weights);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  gather_reduce_kernel<true><<<movement_grid(*d, shape, d->occ_comb, T * p.chunks), kMoveThreads, 0, s>>>(
-      p, static_cast<const uint16_t*>(y), static_cast<uint16_t*>(out));
+  const bool ragged = shape->H % kChunk != 0;
+  const int grid = movement_grid(*d, shape, d->occ_comb[ragged], T * p.chunks);
+  if (ragged)
+    gather_reduce_kernel<true, true><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(y),
+                                                                  static_cast<uint16_t*>(out));
+  else
+    gather_reduce_kernel<true, false><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(y),
+                                                                   static_cast<uint16_t*>(out));
   return finish(handle, s);
 }
 
@@ -358,9 +368,14 @@ int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const voi
   if (T == 0) return EP_OK;
   const MoveParams p = move_params(shape, handle, topk_weights);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  combine_backward_kernel<<<movement_grid(*d, shape, d->occ_cbwd, T * shape->k), kMoveThreads, 0, s>>>(
-      p, static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y), static_cast<uint16_t*>(grad_y),
-      grad_w);
+  const bool ragged = shape->H % kChunk != 0;
+  const int grid = movement_grid(*d, shape, d->occ_cbwd[ragged], T * shape->k);
+  const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
+  const uint16_t* yp = static_cast<const uint16_t*>(y);
+  if (ragged)
+    combine_backward_kernel<true><<<grid, kMoveThreads, 0, s>>>(p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
+  else
+    combine_backward_kernel<false><<<grid, kMoveThreads, 0, s>>>(p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
   return finish(handle, s);
 }
 
@@ -376,8 +391,14 @@ int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv, const e
   if (T == 0) return EP_OK;
   const MoveParams p = move_params(shape, handle, nullptr);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  gather_reduce_kernel<false><<<movement_grid(*d, shape, d->occ_dbwd, T * p.chunks), kMoveThreads, 0, s>>>(
-      p, static_cast<const uint16_t*>(grad_recv), static_cast<uint16_t*>(grad_x));
+  const bool ragged = shape->H % kChunk != 0;
+  const int grid = movement_grid(*d, shape, d->occ_dbwd[ragged], T * p.chunks);
+  if (ragged)
+    gather_reduce_kernel<false, true><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_recv),
+                                                                   static_cast<uint16_t*>(grad_x));
+  else
+    gather_reduce_kernel<false, false><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_recv),
+                                                                    static_cast<uint16_t*>(grad_x));
   return finish(handle, s);
 }
 

@@ -9,12 +9,13 @@
 // section 3.2).
 //
 // All four kernels are HBM-bound streams.  Work unit = one warp x one token x
-// one 512-channel chunk: each lane moves 16 channels (two 16-byte bf16
-// vectors), so a warp reads or writes 1 KiB of bf16 (512 B of E4M3) per row
-// with fully coalesced 16-byte accesses, and an FP8 scale group (128
-// channels) is exactly 8 lanes.  Grids are capped at (SMs x resident CTAs)
-// and stride over the units.  Read-only inputs use non-coherent,
-// L1-no-allocate loads.
+// one 512-channel chunk: each lane moves 16 channels as two 8-channel pieces
+// half a chunk apart (piece_channel), so every 16-byte access of the warp
+// covers 512 contiguous bytes of bf16 (256 of E4M3): 16 sectors per request.
+// A warp reads or writes 1 KiB of bf16 (512 B of E4M3) per row, and an FP8
+// scale group (128 channels) is one half-warp's pieces.  Grids are capped at
+// (SMs x resident CTAs) and stride over the units.  Read-only inputs use
+// non-coherent, L1-no-allocate loads.
 #pragma once
 
 #include "common.cuh"
@@ -35,34 +36,24 @@ constexpr int kMoveWarps = kMoveThreads / kWarp;
 
 // The IEEE-division fallback of quotients_by_scale, out of line: it runs
 // only for groups or elements outside the fast path's range.
-struct Quot16 {
-  float v[16];
+struct Quot8 {
+  float v[8];
 };
 
-__device__ __noinline__ Quot16 quotients_ieee(uint4 v0, uint4 v1, float scale, bool group_fast, Quot16 q) {
-  float f[16];
-  unpack8(v0, f);
-  unpack8(v1, f + 8);
+__device__ __noinline__ Quot8 quotients_ieee(uint4 v, float scale, bool group_fast, Quot8 q) {
+  float f[8];
+  unpack8(v, f);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const uint32_t mag = __float_as_uint(f[i]) & 0x7FFFFFFFu;
     if (!(group_fast && (mag >= 0x0B000000u || mag == 0u))) q.v[i] = __fdiv_rn(f[i], scale);
   }
   return q;
 }
 
-__device__ __forceinline__ void quotients_by_scale_ieee(const uint4& v0, const uint4& v1, float scale,
-                                                        bool group_fast, float* q) {
-  Quot16 in;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) in.v[i] = q[i];
-  const Quot16 out = quotients_ieee(v0, v1, scale, group_fast, in);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) q[i] = out.v[i];
-}
-
-// q[i] <- x_i / scale, rounded to nearest even in fp32, for the 16 values of one
-// 128-channel group (scale >= the group's amax / 448).
+// q[i] <- x_i / scale, rounded to nearest even in fp32, for the 8 values of
+// one piece (scale >= the group's amax / 448).  Every lane of the warp calls
+// it together.
 //
 // Fast path (Markstein's division with a correctly rounded reciprocal, P.
 // Markstein, "Computation of elementary functions on the IBM RISC System/6000
@@ -74,16 +65,14 @@ __device__ __forceinline__ void quotients_by_scale_ieee(const uint4& v0, const u
 // (x, amax) pair of bf16 values was checked: the resulting E4M3 codes equal
 // those of the IEEE division.  Other elements (zeros excepted) take the IEEE
 // division, which a warp executes only if one of its lanes needs it.
-__device__ __forceinline__ void quotients_by_scale(const uint4& v0, const uint4& v1, float scale,
-                                                   float* q) {
-  float f[16];
-  unpack8(v0, f);
-  unpack8(v1, f + 8);
+__device__ __forceinline__ void quotients_by_scale(const uint4& v, float scale, float* q) {
+  float f[8];
+  unpack8(v, f);
   const float r = __frcp_rn(scale);
   const bool group_fast = scale >= 1.17549435e-38f && r <= 3.40282347e+38f;
   bool any_slow = false;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const uint32_t b = __float_as_uint(f[i]);
     const uint32_t mag = b & 0x7FFFFFFFu;
     any_slow |= !(group_fast && (mag >= 0x0B000000u || mag == 0u));
@@ -92,7 +81,37 @@ __device__ __forceinline__ void quotients_by_scale(const uint4& v0, const uint4&
     const float e = fmaf(-q0, scale, ax);
     q[i] = __uint_as_float(__float_as_uint(fmaf(e, r, q0)) | (b & 0x80000000u));
   }
-  if (__any_sync(0xffffffffu, any_slow)) quotients_by_scale_ieee(v0, v1, scale, group_fast, q);
+  if (__any_sync(0xffffffffu, any_slow)) {
+    Quot8 in;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) in.v[i] = q[i];
+    const Quot8 out = quotients_ieee(v, scale, group_fast, in);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) q[i] = out.v[i];
+  }
+}
+
+// Largest |x| of the 128-channel group a piece belongs to: the piece's 8
+// values, then the 16 lanes of the half-warp that hold the group.
+__device__ __forceinline__ float group_amax(const uint4& v) {
+  float f[8];
+  unpack8(v, f);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
+#pragma unroll
+  for (int o = 1; o < kLanesPerGroup; o <<= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  return a;
+}
+
+// The FP8 encoding of one piece: the group's scale (amax / 448, or 1 when
+// amax / 448 is 0) and the 8 E4M3 codes of x / scale.
+__device__ __forceinline__ uint2 quantize_piece(const uint4& v, float& scale) {
+  scale = __fdiv_rn(group_amax(v), kE4M3Max);
+  if (scale == 0.0f) scale = 1.0f;
+  float f[8];
+  quotients_by_scale(v, scale, f);
+  return pack8_e4m3(f);
 }
 
 template <bool FP8>
@@ -105,12 +124,12 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int t = static_cast<int>(u / p.chunks);
     const int c = static_cast<int>(u - static_cast<int64_t>(t) * p.chunks);
-    const int h0 = c * kChunk + lane * kLaneElems;
-    const bool a0 = h0 < p.H, a1 = h0 + 8 < p.H;
-    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H + h0;
+    const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
+    const bool a0 = h0 < p.H, a1 = h1 < p.H;
+    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
     uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-    if (a0) v0 = ld_ro_v4(xr);
-    if (a1) v1 = ld_ro_v4(xr + 8);
+    if (a0) v0 = ld_ro_v4(xr + h0);
+    if (a1) v1 = ld_ro_v4(xr + h1);
     int my_slot = -1;
     float my_w = 0.0f;
     if (lane < p.k) {
@@ -118,37 +137,23 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
       my_w = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
     }
     if constexpr (FP8) {
-      float amax = 0.0f;
-      {
-        float f[16];
-        unpack8(v0, f);
-        unpack8(v1, f + 8);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-      }
-      // 8 consecutive lanes hold one 128-channel group
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-      float scale = __fdiv_rn(amax, kE4M3Max);
-      if (scale == 0.0f) scale = 1.0f;
-      float f[16];
-      quotients_by_scale(v0, v1, scale, f);
-      uint32_t q[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = pack_e4m3x2(f[4 * i + 0], f[4 * i + 1]);
-        const uint32_t hi = pack_e4m3x2(f[4 * i + 2], f[4 * i + 3]);
-        q[i] = lo | (hi << 16);
-      }
-      const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
+      float sc0, sc1;
+      const uint2 q0 = quantize_piece(v0, sc0);
+      const uint2 q1 = quantize_piece(v1, sc1);
+      const bool scale_lane = (lane & (kLanesPerGroup - 1)) == 0;
       uint8_t* rx = static_cast<uint8_t*>(recv_x);
       for (int j = 0; j < p.k; ++j) {
         const int s = __shfl_sync(0xffffffffu, my_slot, j);
-        if (s >= 0 && a0) {
-          st_v4(rx + static_cast<int64_t>(s) * p.H + h0, qv);
-          if ((lane & (kLanesPerGroup - 1)) == 0)
-            recv_scale[static_cast<int64_t>(s) * p.G + h0 / kGroup] = scale;
+        if (s < 0) continue;
+        uint8_t* row = rx + static_cast<int64_t>(s) * p.H;
+        float* srow = recv_scale + static_cast<int64_t>(s) * p.G;
+        if (a0) {
+          *reinterpret_cast<uint2*>(row + h0) = q0;
+          if (scale_lane) srow[h0 / kGroup] = sc0;
+        }
+        if (a1) {
+          *reinterpret_cast<uint2*>(row + h1) = q1;
+          if (scale_lane) srow[h1 / kGroup] = sc1;
         }
       }
     } else {
@@ -156,9 +161,9 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
       for (int j = 0; j < p.k; ++j) {
         const int s = __shfl_sync(0xffffffffu, my_slot, j);
         if (s >= 0) {
-          uint16_t* dst = rx + static_cast<int64_t>(s) * p.H + h0;
-          if (a0) st_v4(dst, v0);
-          if (a1) st_v4(dst + 8, v1);
+          uint16_t* row = rx + static_cast<int64_t>(s) * p.H;
+          if (a0) st_v4(row + h0, v0);
+          if (a1) st_v4(row + h1, v1);
         }
       }
     }
@@ -226,16 +231,16 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
   extern __shared__ __align__(128) uint8_t tma_smem[];
   const TmaSmemLayout L = tma_smem_layout(p.H, FP8);
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
-  const int h0 = warp * kChunk + lane * kLaneElems;  // one chunk per warp
-  const bool a0 = h0 < p.H, a1 = h0 + 8 < p.H;
+  const int h0 = piece_channel(warp, lane), h1 = h0 + kHalfChunk;  // one chunk per warp
+  const bool a0 = h0 < p.H, a1 = h1 < p.H;
   const int row_bytes = FP8 ? p.H : 2 * p.H;
 
   uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
   int t = blockIdx.x;
   if (t < p.T) {
-    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H + h0;
-    if (a0) v0 = ld_ro_v4(xr);
-    if (a1) v1 = ld_ro_v4(xr + 8);
+    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
+    if (a0) v0 = ld_ro_v4(xr + h0);
+    if (a1) v1 = ld_ro_v4(xr + h1);
   }
   for (int it = 0; t < p.T; ++it, t += gridDim.x) {
     const int stage = it & 1;
@@ -248,9 +253,9 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
     const int tn = t + gridDim.x;
     uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
     if (tn < p.T) {
-      const uint16_t* xr = x + static_cast<int64_t>(tn) * p.H + h0;
-      if (a0) n0 = ld_ro_v4(xr);
-      if (a1) n1 = ld_ro_v4(xr + 8);
+      const uint16_t* xr = x + static_cast<int64_t>(tn) * p.H;
+      if (a0) n0 = ld_ro_v4(xr + h0);
+      if (a1) n1 = ld_ro_v4(xr + h1);
     }
     // the row stage is free once the copies issued L.stages tokens ago have read it
     if (threadIdx.x == 0) bulk_wait_read_all_but(L.stages - 1);
@@ -261,32 +266,21 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
     __syncthreads();
 
     if constexpr (FP8) {
-      float amax = 0.0f;
-      {
-        float f[16];
-        unpack8(v0, f);
-        unpack8(v1, f + 8);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-      }
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-      float scale = __fdiv_rn(amax, kE4M3Max);
-      if (scale == 0.0f) scale = 1.0f;
-      float f[16];
-      quotients_by_scale(v0, v1, scale, f);
-      uint32_t q[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        q[i] = pack_e4m3x2(f[4 * i + 0], f[4 * i + 1]) | (pack_e4m3x2(f[4 * i + 2], f[4 * i + 3]) << 16);
+      float sc0, sc1;
+      const uint2 q0 = quantize_piece(v0, sc0);
+      const uint2 q1 = quantize_piece(v1, sc1);
+      const bool scale_lane = (lane & (kLanesPerGroup - 1)) == 0;
       if (a0) {
-        *reinterpret_cast<uint4*>(row + h0) = make_uint4(q[0], q[1], q[2], q[3]);
-        if ((lane & (kLanesPerGroup - 1)) == 0) sscale[h0 / kGroup] = scale;
+        *reinterpret_cast<uint2*>(row + h0) = q0;
+        if (scale_lane) sscale[h0 / kGroup] = sc0;
+      }
+      if (a1) {
+        *reinterpret_cast<uint2*>(row + h1) = q1;
+        if (scale_lane) sscale[h1 / kGroup] = sc1;
       }
     } else {
       if (a0) *reinterpret_cast<uint4*>(row + 2 * h0) = v0;
-      if (a1) *reinterpret_cast<uint4*>(row + 2 * h0 + 16) = v1;
+      if (a1) *reinterpret_cast<uint4*>(row + 2 * h1) = v1;
     }
     // make the generic-proxy shared-memory writes visible to the bulk copies
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -324,7 +318,11 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
 // with acc = +0.0f and j = 0..k-1 in order.  The k rows are fetched in
 // batches of 8 (all loads of a batch issued before the arithmetic).
 
-template <bool WEIGHTED>
+// RAGGED (H not a multiple of 512): every piece is checked against H.
+// Otherwise every piece lies inside the row and no check is made; a kernel
+// that carries both paths was measured slower even on full chunks, so the
+// host launches the variant the shape needs.
+template <bool WEIGHTED, bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __restrict__ out) {
   const int lane = threadIdx.x & (kWarp - 1);
@@ -333,8 +331,8 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int t = static_cast<int>(u / p.chunks);
     const int c = static_cast<int>(u - static_cast<int64_t>(t) * p.chunks);
-    const int h0 = c * kChunk + lane * kLaneElems;
-    const bool a0 = h0 < p.H, a1 = h0 + 8 < p.H;
+    const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
+    const bool a0 = !RAGGED || h0 < p.H, a1 = !RAGGED || h1 < p.H;
     int my_slot = -1;
     float my_w = 0.0f;
     if (lane < p.k) {
@@ -360,9 +358,9 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
         v[jj][0] = make_uint4(0, 0, 0, 0);
         v[jj][1] = v[jj][0];
         if (s[jj] >= 0) {
-          const uint16_t* src = y + static_cast<int64_t>(s[jj]) * p.H + h0;
-          if (a0) v[jj][0] = ld_ro_v4(src);
-          if (a1) v[jj][1] = ld_ro_v4(src + 8);
+          const uint16_t* src = y + static_cast<int64_t>(s[jj]) * p.H;
+          if (a0) v[jj][0] = ld_ro_v4(src + h0);
+          if (a1) v[jj][1] = ld_ro_v4(src + h1);
         }
       }
 #pragma unroll
@@ -379,9 +377,9 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
         }
       }
     }
-    uint16_t* dst = out + static_cast<int64_t>(t) * p.H + h0;
-    if (a0) st_v4(dst, pack8_bf16(acc));
-    if (a1) st_v4(dst + 8, pack8_bf16(acc + 8));
+    uint16_t* dst = out + static_cast<int64_t>(t) * p.H;
+    if (a0) st_v4(dst + h0, pack8_bf16(acc));
+    if (a1) st_v4(dst + h1, pack8_bf16(acc + 8));
   }
 }
 
@@ -403,6 +401,10 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
 constexpr int kCbwdUnroll = 4;
 static_assert(kCbwdUnroll == 4, "the partial sums below are added as two pairs");
 
+// RAGGED (H not a multiple of 512): every piece is checked against H;
+// otherwise one check per chunk covers both pieces (6 % faster than
+// checking each piece, and the host launches the variant the shape needs).
+template <bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 combine_backward_kernel(MoveParams p, const uint16_t* __restrict__ g, const uint16_t* __restrict__ y,
                         uint16_t* __restrict__ grad_y, float* __restrict__ grad_w) {
@@ -428,20 +430,22 @@ combine_backward_kernel(MoveParams p, const uint16_t* __restrict__ g, const uint
       uint4 gv[kCbwdUnroll][2], yv[kCbwdUnroll][2];
 #pragma unroll
       for (int q = 0; q < kCbwdUnroll; ++q) {
-        const int h0 = (c0 + q) * kChunk + lane * kLaneElems;
+        const int h0 = piece_channel(c0 + q, lane), h1 = h0 + kHalfChunk;
         gv[q][0] = gv[q][1] = yv[q][0] = yv[q][1] = make_uint4(0, 0, 0, 0);
-        if (h0 < p.H) {
-          gv[q][0] = ld_l1_v4(gr + h0);
-          yv[q][0] = ld_ro_v4(yr + h0);
-        }
-        if (h0 + 8 < p.H) {
-          gv[q][1] = ld_l1_v4(gr + h0 + 8);
-          yv[q][1] = ld_ro_v4(yr + h0 + 8);
+        if (c0 + q < p.chunks) {
+          if (!RAGGED || h0 < p.H) {
+            gv[q][0] = ld_l1_v4(gr + h0);
+            yv[q][0] = ld_ro_v4(yr + h0);
+          }
+          if (!RAGGED || h1 < p.H) {
+            gv[q][1] = ld_l1_v4(gr + h1);
+            yv[q][1] = ld_ro_v4(yr + h1);
+          }
         }
       }
 #pragma unroll
       for (int q = 0; q < kCbwdUnroll; ++q) {
-        const int h0 = (c0 + q) * kChunk + lane * kLaneElems;
+        const int h0 = piece_channel(c0 + q, lane), h1 = h0 + kHalfChunk;
         uint4 out[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -457,8 +461,10 @@ combine_backward_kernel(MoveParams p, const uint16_t* __restrict__ g, const uint
           }
           out[h] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        if (h0 < p.H) st_v4_hint(dr + h0, out[0], evict_first);
-        if (h0 + 8 < p.H) st_v4_hint(dr + h0 + 8, out[1], evict_first);
+        if (c0 + q < p.chunks) {
+          if (!RAGGED || h0 < p.H) st_v4_hint(dr + h0, out[0], evict_first);
+          if (!RAGGED || h1 < p.H) st_v4_hint(dr + h1, out[1], evict_first);
+        }
       }
     }
     float dot = (d[0] + d[1]) + (d[2] + d[3]);
