@@ -258,15 +258,30 @@ def launches_per_step(w) -> int:
     return (1 if small else 3) + 4
 
 
-def bench_config(w, args, world: int) -> dict:
+B200_L2_BYTES = 126 * 2**20
+
+
+def l2_policy(step_bytes: int, l2_bytes: int) -> tuple:
+    """(flush, description): no flush when a step moves at least 4x the L2
+    size, so that no buffer is still in L2 when the next step reads it;
+    otherwise L2 is flushed before every timed step."""
+    if step_bytes >= 4 * l2_bytes:
+        return False, (f"no flush: a step moves {step_bytes / 1e6:.0f} MB, {step_bytes / l2_bytes:.0f}x the "
+                       f"{l2_bytes / 2**20:.0f} MiB L2, so no buffer is still in L2 when the next step reads it")
+    return True, (f"L2 flushed before every step ({2 * l2_bytes / 2**20:.0f} MiB written outside the timed "
+                  f"region; each step timed on its own)")
+
+
+def bench_config(w, args, world: int, l2_bytes: int = B200_L2_BYTES) -> dict:
     """The JSON line's config: the workload by name and sizes (both arms)."""
+    step_bytes = sum(call_bytes(w)[c] for c in step_calls(args))
     return {"workload": f"{w.name}: T={w.T} ({w.R} virtual ranks x {w.T // w.R} tokens), H={w.H}, "
                         f"E={w.E}, k={w.k}, top-{w.topk_groups} of {w.n_groups} groups, "
                         f"{'FP8' if w.use_fp8 else 'BF16'} dispatch + BF16 combine + both backward passes",
             "T": w.T, "H": w.H, "k": w.k, "E": w.E, "R": w.R, "use_fp8": w.use_fp8,
             "storage": ("e4m3 codes + f32 scales dispatched, bf16 expert rows, outputs and gradients"
                         if w.use_fp8 else "bf16 rows, outputs and gradients"),
-            "step_bytes": sum(call_bytes(w)[c] for c in step_calls(args)), "l2": "inputs larger than L2 (no flush)",
+            "step_bytes": step_bytes, "l2": l2_policy(step_bytes, l2_bytes)[1],
             "receive_layout": (f"padded [E][R][{args.max_tokens_per_rank}]" if args.max_tokens_per_rank
                                else "dense [T*k]"),
             "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, virtual ranks",
@@ -292,6 +307,13 @@ def run_ours(args, rank, world, local):
     nb = {c: v for c, v in call_bytes(w).items() if c in calls}
     step_bytes = sum(nb.values())
     nmarks = len(calls) + 1
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size or B200_L2_BYTES
+    flush, _ = l2_policy(step_bytes, l2_bytes)
+    flush_buf = torch.empty(2 * l2_bytes // 4, dtype=torch.int32, device=dev) if flush else None
+
+    def flush_l2(i: int):
+        if flush_buf is not None:
+            flush_buf.fill_(i)
 
     def barrier():
         torch.cuda.synchronize()
@@ -318,7 +340,8 @@ def run_ours(args, rank, world, local):
         for _ in range(args.warmup):
             run_step()
         # per-call breakdown: one replay at a time, events read after each
-        for _ in range(min(args.steps, 20)):
+        for i in range(min(args.steps, 20)):
+            flush_l2(i)
             run_step()
             torch.cuda.synchronize()
             for ci, c in enumerate(calls):
@@ -331,13 +354,20 @@ def run_ours(args, rank, world, local):
     sampler = ClockSampler(local)
     sampler.start()
     barrier()
+    step_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)] if flush else []
     t0 = time.time()
     e_start.record()
     for s in range(args.steps):
+        if flush:  # the flush stays outside the per-step events
+            flush_l2(s)
+            step_events[s][0].record()
         if args.no_graph:
             path.step(marks[s])
         else:
             run_step()
+        if flush:
+            step_events[s][1].record()
     e_end.record()
     torch.cuda.synchronize()
     t1 = time.time()
@@ -348,7 +378,8 @@ def run_ours(args, rank, world, local):
         for m in marks:
             for ci, c in enumerate(calls):
                 per_call_ms[c].append(m[ci].elapsed_time(m[ci + 1]))
-    total_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
+    local_ms = (sum(a.elapsed_time(b) for a, b in step_events) if flush else e_start.elapsed_time(e_end))
+    total_ms = max_over_ranks(local_ms, world, dev)
     ms_per_step = total_ms / args.steps
 
     # End to end through the same C ABI: every step copies its inputs from
@@ -459,7 +490,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded group-limited routing, N(0,1) activations)",
-        "config": bench_config(w, args, world),
+        "config": bench_config(w, args, world, l2_bytes),
         "per_call": per_call,
         "roofline": {"kernel": kernel_of[dominant], "call": dominant, "bound": "hbm", "achieved": ach,
                      "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 3),
