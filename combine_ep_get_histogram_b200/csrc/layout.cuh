@@ -331,6 +331,7 @@ layout_small_kernel(LayoutParams p) {
   const int64_t pair0 = static_cast<int64_t>(t0) * p.k;
   const int S = ((npairs + kSmallWarps - 1) / kSmallWarps + kWarp - 1) / kWarp * kWarp;
   const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
+  const int my_chunks = my_hi > my_lo ? (my_hi - my_lo + kWarp - 1) / kWarp : 0;  // chunks holding pairs (warp-uniform)
 
   bool bad = false;
   int ereg[kSmallChunks];
@@ -348,6 +349,7 @@ layout_small_kernel(LayoutParams p) {
   int32_t* wh = whist + warp * p.E;
 #pragma unroll
   for (int q = 0; q < kSmallChunks; ++q) {
+    if (q >= my_chunks) break;
     const int i = my_lo + q * kWarp + lane;
     const int e = ereg[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
@@ -403,6 +405,7 @@ layout_small_kernel(LayoutParams p) {
   const uint32_t lt = lanemask_lt();
 #pragma unroll
   for (int q = 0; q < kSmallChunks; ++q) {
+    if (q >= my_chunks) break;
     const int i = my_lo + q * kWarp + lane;
     const int e = ereg[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
@@ -495,6 +498,7 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
   const int64_t pair0 = static_cast<int64_t>(r) * p.Tr * p.k;
   const int S = ((npairs + kPadWarps - 1) / kPadWarps + kWarp - 1) / kWarp * kWarp;
   const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
+  const int my_chunks = my_hi > my_lo ? (my_hi - my_lo + kWarp - 1) / kWarp : 0;  // chunks holding pairs (warp-uniform)
 
   bool bad = false, over = false;
   int ereg[kPadChunks];
@@ -510,6 +514,7 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
   int32_t* wh = whist + warp * p.E;
 #pragma unroll
   for (int q = 0; q < kPadChunks; ++q) {
+    if (q >= my_chunks) break;
     const int i = my_lo + q * kWarp + lane;
     const int e = ereg[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
@@ -537,6 +542,7 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
   const uint32_t lt = lanemask_lt();
 #pragma unroll
   for (int q = 0; q < kPadChunks; ++q) {
+    if (q >= my_chunks) break;
     const int i = my_lo + q * kWarp + lane;
     const int e = ereg[q];
     const unsigned same = __match_any_sync(0xffffffffu, e);
