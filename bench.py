@@ -62,19 +62,34 @@ def call_bytes(w) -> dict:
 MEASURED_TRAFFIC = {
     ("prefill", 32768, "combine_backward"): {
         "bytes": 4.23e9 + 3.70e9,
-        "sources_sha1": "316cb20ce7f2826bc350f919968a031502262857",
+        "sources_sha1": "3ad17ff065069ece68cd7402e219ae70395a65c5",
     },
 }
 KERNEL_SOURCES = ("combine_ep_get_histogram_b200/csrc/common.cuh",
                   "combine_ep_get_histogram_b200/csrc/movement.cuh")
 
 
-def kernel_sources_sha1() -> str:
+def code_lines(text: str) -> str:
+    """The source without // comments, trailing blanks and blank lines, so
+    that a comment edit leaves the hash of the code unchanged."""
+    out = []
+    for line in text.splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code:
+            out.append(code)
+    return "\n".join(out)
+
+
+def kernel_sources_sha1(read=None) -> str:
     import hashlib
     h = hashlib.sha1()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        if read is None:
+            with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+                text = fh.read()
+        else:
+            text = read(f)
+        h.update(code_lines(text).encode())
     return h.hexdigest()
 
 

@@ -387,7 +387,7 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
 //
 // One warp per (token t, top-k position j) pair, grid-stride over the pairs:
 // the warp streams the whole y[slot] row in and the whole grad_y[slot] row
-// out, kUnroll 512-channel chunks at a time, and reads g[t] through L1 (the
+// out, kCbwdUnroll 512-channel chunks at a time, and reads g[t] through L1 (the
 // k warps of one token usually share a CTA, so g comes from DRAM once).
 // grad_y = bf16(w * g) (one fp32 product).  The dot product g . y[slot]
 // keeps kCbwdUnroll fp32 partial sums per lane, one per chunk slot of an

@@ -1,0 +1,46 @@
+"""Host-side helpers of bench.py that need no GPU: the code hash that keeps a
+measured DRAM-traffic figure tied to the kernel it was taken on, and the L2
+statement made from a step's bytes."""
+
+import os
+
+import bench
+
+
+def _reader(edit=None):
+    def read(f):
+        with open(os.path.join(bench.ROOT, f), encoding="utf-8") as fh:
+            text = fh.read()
+        return edit(f, text) if edit else text
+    return read
+
+
+def test_comment_edits_keep_the_code_hash():
+    base = bench.kernel_sources_sha1(_reader())
+    assert base == bench.kernel_sources_sha1()
+    commented = bench.kernel_sources_sha1(_reader(lambda f, t: t.replace("\n", "  // note\n\n", 3) + "// end\n"))
+    assert commented == base
+
+
+def test_code_edits_change_the_code_hash():
+    base = bench.kernel_sources_sha1()
+    edited = bench.kernel_sources_sha1(_reader(lambda f, t: t + "\nconstexpr int kUnused = 1;\n"
+                                               if f.endswith("movement.cuh") else t))
+    assert edited != base
+
+
+def test_traffic_is_reported_only_for_the_captured_code():
+    from combine_ep_get_histogram_b200 import workloads as wl
+    w = wl.CONFIGS["prefill"]
+    entry = bench.MEASURED_TRAFFIC[(w.name, w.T, "combine_backward")]
+    expect = entry["bytes"] if entry["sources_sha1"] == bench.kernel_sources_sha1() else None
+    assert bench.measured_traffic(w, "combine_backward") == expect
+    assert bench.measured_traffic(w, "dispatch") is None
+
+
+def test_l2_statement_follows_the_step_bytes():
+    l2 = 126 * 2**20
+    flush, text = bench.l2_policy(4 * l2, l2)
+    assert not flush and "no flush" in text
+    flush, text = bench.l2_policy(4 * l2 - 1, l2)
+    assert flush and "flushed" in text
