@@ -265,12 +265,70 @@ class Path:
         rec()
 
 
-def launches_per_step(w) -> int:
+def launches_per_step(w, peers: bool = False) -> int:
     """Kernels one step launches: layout (one kernel for small problems, else
-    count + scan + assign), dispatch, combine and the two backward passes."""
+    count + scan + assign), dispatch, combine and the two backward passes
+    (once per rank with the peer calls)."""
     small = (w.T * w.k <= 16384 and w.E <= 256 and w.R <= 64 and w.R * w.E <= 2048
              and -(-w.T // 8) * w.R <= 8192)
-    return (1 if small else 3) + 4
+    return (1 if small else 3) + 4 * (w.R if peers else 1)
+
+
+class PeersPath(Path):
+    """The step of multi-GPU expert parallelism with its R ranks emulated on
+    one GPU: one global layout, then every rank's peer calls for its own
+    tokens, each owner rank's receive buffers a separate allocation."""
+
+    def __init__(self, w, d, dev):
+        import torch
+        super().__init__(w, d, dev)
+        ep, multi = self.ep, __import__("combine_ep_get_histogram_b200.multi", fromlist=["multi"])
+        ep.ep_get_dispatch_layout(self.shape, self.inp["topk_idx"], self.handle, self.ws)
+        torch.cuda.synchronize()
+        rows = multi.owner_rows(self.handle.tensors["expert_offset"].cpu().numpy(), w.E, w.R)
+        pay = torch.uint8 if w.use_fp8 else torch.int16
+
+        def bufs(cols, dtype):
+            return [torch.empty((max(n, 1),) + cols, dtype=dtype, device=dev) for _, n in rows]
+
+        self.rx, self.rw, self.gy = bufs((w.H,), pay), bufs((), torch.float32), bufs((w.H,), torch.int16)
+        self.rs = bufs((w.G,), torch.float32) if w.use_fp8 else None
+        self.ys = [self.inp["y"][r0:r0 + n] if n else torch.empty((1, w.H), dtype=torch.int16, device=dev)
+                   for r0, n in rows]
+        Tl = w.T // w.R
+        self.ranks = [(r, slice(r * Tl, (r + 1) * Tl)) for r in range(w.R)]
+
+    def step(self, marks=None, before_back=None, after_combine=None):
+        ep, i, sh, h = self.ep, self.inp, self.shape, self.handle
+        n = 0
+
+        def rec():
+            nonlocal n
+            if marks is not None:
+                marks[n].record()
+            n += 1
+
+        rec()
+        ep.ep_get_dispatch_layout(sh, i["topk_idx"], h, self.ws)
+        rec()
+        for r, tok in self.ranks:
+            ep.ep_dispatch_peers(sh, r, i["topk_idx"], h, i["x"][tok], i["topk_weights"][tok], self.rx, self.rs,
+                                 self.rw)
+        rec()
+        if before_back is not None:
+            before_back()
+        for r, tok in self.ranks:
+            ep.ep_combine_peers(sh, r, i["topk_idx"], h, self.ys, i["topk_weights"][tok], self.out[tok])
+        if after_combine is not None:
+            after_combine()
+        rec()
+        for r, tok in self.ranks:
+            ep.ep_combine_backward_peers(sh, r, i["topk_idx"], h, i["g"][tok], self.ys, i["topk_weights"][tok],
+                                         self.gy, self.grad_w[tok])
+        rec()
+        for r, tok in self.ranks:
+            ep.ep_dispatch_backward_peers(sh, r, i["topk_idx"], h, self.gy, self.grad_x[tok])
+        rec()
 
 
 B200_L2_BYTES = 126 * 2**20
@@ -299,7 +357,9 @@ def bench_config(w, args, world: int, l2_bytes: int = B200_L2_BYTES) -> dict:
             "step_bytes": step_bytes, "l2": l2_policy(step_bytes, l2_bytes)[1],
             "receive_layout": (f"padded [E][R][{args.max_tokens_per_rank}]" if args.max_tokens_per_rank
                                else "dense [T*k]"),
-            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU, virtual ranks",
+            "parallelism": (f"replicas x{world}" if world > 1 else
+                            f"1 GPU, {w.R} ranks emulated through the peer-table calls"
+                            if getattr(args, "peers", False) else "1 GPU, virtual ranks"),
             "router_in_step": bool(args.route)}
 
 
@@ -317,7 +377,9 @@ def run_ours(args, rank, world, local):
     d = wl.make_inputs(w, parts=("routing", "x", "g") + (() if M else ("y",)) + (("scores",) if args.route else ()))
     if M:  # expert outputs fill the padded receive rows
         d["y"] = wl.normal_bf16(w.E * w.R * M, w.H, w.seed, 2)
-    path = Path(w, d, dev, M, route=args.route)
+    if args.peers and (M or args.route):
+        raise SystemExit("--peers runs the dense layout without routing")
+    path = PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route)
     stream = torch.cuda.current_stream()
     nb = {c: v for c, v in call_bytes(w).items() if c in calls}
     step_bytes = sum(nb.values())
@@ -404,7 +466,7 @@ def run_ours(args, rank, world, local):
     # third stream; PCIe is full duplex).
     e2e = None
     if not args.no_e2e:
-        paths = [path, Path(w, d, dev, M, route=args.route)]
+        paths = [path, PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route)]
         pin = {n: t.pin_memory() for n, t in path.host.items()}
         outs = {"out": torch.empty_like(path.out, device="cpu").pin_memory(),
                 "grad_x": torch.empty_like(path.grad_x, device="cpu").pin_memory(),
@@ -513,7 +575,7 @@ def run_ours(args, rank, world, local):
                      "bytes_per_launch": nb[dominant], "traffic": measured_traffic(w, dominant),
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, full-size launch"},
         "clocks": clocks,
-        "gpu_launches": (launches_per_step(w) + (1 if args.route else 0)) * args.steps,
+        "gpu_launches": (launches_per_step(w, args.peers) + (1 if args.route else 0)) * args.steps,
         "timing": "CUDA graph replay of the step" if not args.no_graph else "eager launches",
         "e2e": e2e,
     }
@@ -690,6 +752,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each call eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--peers", action="store_true",
+                    help="the step as R ranks emulated on one GPU through the multi-GPU (peer-table) calls")
     ap.add_argument("--overlap-sms", type=int, default=0,
                     help="also time the path with this SM budget on a side stream beside a bf16 GEMM")
     ap.add_argument("--cpu-tokens-per-rank", type=int, default=1536)

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libep_b200.so")
 SOURCES = ["ep_api.cu", "ep_noalloc.cu"]
-DEPS = ["common.cuh", "layout.cuh", "movement.cuh", "route.cuh"]
+DEPS = ["common.cuh", "layout.cuh", "movement.cuh", "peers.cuh", "route.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

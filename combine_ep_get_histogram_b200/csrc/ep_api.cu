@@ -11,6 +11,7 @@
 #include "ep.h"
 #include "layout.cuh"
 #include "movement.cuh"
+#include "peers.cuh"
 #include "route.cuh"
 
 namespace {
@@ -43,6 +44,7 @@ struct DeviceInfo {
   int occ_comb[2] = {}, occ_dbwd[2] = {};  // [ragged]
   int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
   int occ_cbwd[2] = {};  // [ragged]
+  int occ_peer_disp[2] = {}, occ_peer_gather[2] = {}, occ_peer_cbwd = 0;  // [fp8], [weighted]
   int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
   int occ_route_aligned[6] = {};  // route_aligned_kernel<1, 2, 4, 8, 16, 32>
 };
@@ -84,6 +86,13 @@ int device_info(const DeviceInfo** out) {
       d.occ_dbwd[1] = occupancy(reinterpret_cast<const void*>(gather_reduce_kernel<false, true>), kMoveThreads, 0);
       d.occ_cbwd[0] = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<false>), kMoveThreads, 0);
       d.occ_cbwd[1] = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<true>), kMoveThreads, 0);
+      d.occ_peer_disp[0] = occupancy(reinterpret_cast<const void*>(dispatch_peers_kernel<false>), kMoveThreads, 0);
+      d.occ_peer_disp[1] = occupancy(reinterpret_cast<const void*>(dispatch_peers_kernel<true>), kMoveThreads, 0);
+      d.occ_peer_gather[0] =
+          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<false>), kMoveThreads, 0);
+      d.occ_peer_gather[1] =
+          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<true>), kMoveThreads, 0);
+      d.occ_peer_cbwd = occupancy(reinterpret_cast<const void*>(combine_backward_peers_kernel), kMoveThreads, 0);
       const void* route_fns[6] = {reinterpret_cast<const void*>(route_group_limited_kernel<1>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<2>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<4>),
@@ -202,6 +211,48 @@ int movement_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t uni
   const int64_t need = ceil_div(units_per_warp_grid, kMoveWarps);
   const int64_t cap = grid_cap(d, s, occ);
   return static_cast<int>(need < cap ? need : cap);
+}
+
+static_assert(EP_MAX_PEERS == kMaxPeers, "peer tables of the C ABI and the kernels agree");
+
+// Every owner's buffer given, non-null and aligned to `align` bytes.
+bool peer_rows_ok(const ep_peer_rows_t* t, int R, size_t align) {
+  if (t == nullptr) return false;
+  for (int o = 0; o < R; ++o)
+    if (t->rows[o] == nullptr || !aligned(t->rows[o], align)) return false;
+  return true;
+}
+
+PeerRows peer_rows(const ep_peer_rows_t* t) {
+  PeerRows r{};
+  if (t != nullptr)
+    for (int o = 0; o < kMaxPeers; ++o) r.base[o] = t->rows[o];
+  return r;
+}
+
+// Checks common to the peer calls and the kernel parameters of this rank.
+int peer_setup(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, const ep_handle_t* handle,
+               const float* topk_weights, PeerParams* p) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  if (shape->max_tokens_per_rank != 0 || shape->R > EP_MAX_PEERS || rank < 0 || rank >= shape->R)
+    return EP_ERR_INVALID_ARG;
+  const int64_t T = shape->T, Tl = T / shape->R;
+  if (T > 0 && (topk_idx == nullptr || !aligned(topk_idx, 8))) return EP_ERR_INVALID_ARG;
+  if (topk_weights != nullptr && !f32_ok(topk_weights, Tl * shape->k)) return EP_ERR_INVALID_ARG;
+  p->T = static_cast<int>(Tl);
+  p->H = shape->H;
+  p->k = shape->k;
+  p->G = shape->H / kGroup;
+  p->chunks = static_cast<int>(ceil_div(shape->H, kChunk));
+  p->t_begin = static_cast<int>(rank * Tl);
+  p->Er = shape->E / shape->R;
+  p->slot_of_pair = handle->slot_of_pair;
+  p->topk_idx = topk_idx;
+  p->expert_offset = handle->expert_offset;
+  p->topk_weights = topk_weights;
+  return EP_OK;
 }
 
 }  // namespace
@@ -449,6 +500,88 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
     default: route_group_limited_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
   }
   return cuda_status(cudaGetLastError());
+}
+
+int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, const ep_handle_t* handle,
+                      const void* x, const float* topk_weights, const ep_peer_rows_t* recv_x,
+                      const ep_peer_rows_t* recv_scale, const ep_peer_rows_t* recv_weight, ep_stream_t stream) {
+  PeerParams p;
+  const DeviceInfo* d = nullptr;
+  int st = peer_setup(shape, rank, topk_idx, handle, topk_weights, &p);
+  if (st != EP_OK) return st;
+  if (topk_weights == nullptr && p.T > 0) return EP_ERR_INVALID_ARG;
+  const int R = shape->R;
+  if (!rows_ok(x, p.T) || (p.T > 0 && !peer_rows_ok(recv_x, R, 16))) return EP_ERR_INVALID_ARG;
+  if (shape->use_fp8 && p.T > 0 && !peer_rows_ok(recv_scale, R, 4)) return EP_ERR_INVALID_ARG;
+  if (recv_weight != nullptr && p.T > 0 && !peer_rows_ok(recv_weight, R, 4)) return EP_ERR_INVALID_ARG;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (p.T == 0) return EP_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t units = static_cast<int64_t>(p.T) * p.chunks;
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  const PeerRows rx = peer_rows(recv_x), rs = peer_rows(recv_scale), rw = peer_rows(recv_weight);
+  if (shape->use_fp8)
+    dispatch_peers_kernel<true><<<movement_grid(*d, shape, d->occ_peer_disp[1], units), kMoveThreads, 0, s>>>(
+        p, xs, rx, rs, rw);
+  else
+    dispatch_peers_kernel<false><<<movement_grid(*d, shape, d->occ_peer_disp[0], units), kMoveThreads, 0, s>>>(
+        p, xs, rx, rs, rw);
+  return finish(handle, s);
+}
+
+int ep_combine_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, const ep_handle_t* handle,
+                     const ep_peer_rows_t* y, const float* topk_weights, void* out, ep_stream_t stream) {
+  PeerParams p;
+  const DeviceInfo* d = nullptr;
+  int st = peer_setup(shape, rank, topk_idx, handle, topk_weights, &p);
+  if (st != EP_OK) return st;
+  if (topk_weights == nullptr && p.T > 0) return EP_ERR_INVALID_ARG;
+  if (!rows_ok(out, p.T) || (p.T > 0 && !peer_rows_ok(y, shape->R, 16))) return EP_ERR_INVALID_ARG;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (p.T == 0) return EP_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int grid = movement_grid(*d, shape, d->occ_peer_gather[1], static_cast<int64_t>(p.T) * p.chunks);
+  gather_reduce_peers_kernel<true><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(y), static_cast<uint16_t*>(out));
+  return finish(handle, s);
+}
+
+int ep_combine_backward_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx,
+                              const ep_handle_t* handle, const void* grad_out, const ep_peer_rows_t* y,
+                              const float* topk_weights, const ep_peer_rows_t* grad_y, float* grad_w,
+                              ep_stream_t stream) {
+  PeerParams p;
+  const DeviceInfo* d = nullptr;
+  int st = peer_setup(shape, rank, topk_idx, handle, topk_weights, &p);
+  if (st != EP_OK) return st;
+  if (topk_weights == nullptr && p.T > 0) return EP_ERR_INVALID_ARG;
+  const int R = shape->R;
+  if (!rows_ok(grad_out, p.T) || !f32_ok(grad_w, static_cast<int64_t>(p.T) * p.k) ||
+      (p.T > 0 && (!peer_rows_ok(y, R, 16) || !peer_rows_ok(grad_y, R, 16))))
+    return EP_ERR_INVALID_ARG;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (p.T == 0) return EP_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int grid = movement_grid(*d, shape, d->occ_peer_cbwd, static_cast<int64_t>(p.T) * p.k);
+  combine_backward_peers_kernel<<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_out),
+                                                             peer_rows(y), peer_rows(grad_y), grad_w);
+  return finish(handle, s);
+}
+
+int ep_dispatch_backward_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx,
+                               const ep_handle_t* handle, const ep_peer_rows_t* grad_recv, void* grad_x,
+                               ep_stream_t stream) {
+  PeerParams p;
+  const DeviceInfo* d = nullptr;
+  int st = peer_setup(shape, rank, topk_idx, handle, nullptr, &p);
+  if (st != EP_OK) return st;
+  if (!rows_ok(grad_x, p.T) || (p.T > 0 && !peer_rows_ok(grad_recv, shape->R, 16))) return EP_ERR_INVALID_ARG;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  if (p.T == 0) return EP_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int grid = movement_grid(*d, shape, d->occ_peer_gather[0], static_cast<int64_t>(p.T) * p.chunks);
+  gather_reduce_peers_kernel<false><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(grad_recv),
+                                                                 static_cast<uint16_t*>(grad_x));
+  return finish(handle, s);
 }
 
 int ep_get_error(const ep_handle_t* handle, ep_stream_t stream) {

@@ -1,0 +1,221 @@
+// Multi-GPU expert parallelism: the data-movement kernels of one rank, with
+// every receive-side row in its owner rank's buffer.
+//
+// One process per GPU.  Rank r holds tokens [r*T/R, (r+1)*T/R) and experts
+// [r*E/R, (r+1)*E/R).  Every rank has all ranks' expert ids and has run the
+// same layout over them, so slots are global: the pair (t, j) to expert e
+// takes slot s in e's block, exactly as on one GPU.  The owner o = e / (E/R)
+// keeps the rows [expert_offset[o*E/R], expert_offset[(o+1)*E/R]) of the
+// global receive buffer, and slot s is its local row s - expert_offset[o*E/R].
+// The kernels fuse the exchange with the arithmetic (the pages' dispatch and
+// combine are all-to-alls between ranks: zhouruolin.cn, section 五; the
+// normal kernels move tokens over NVLink: blog.hotdry.top, section 一).
+// Dispatch quantises this rank's tokens and stores each row straight into
+// its owner's buffer.  Combine and dispatch backward load the owners' rows
+// and reduce them.  Combine backward loads y from, and stores grad_y into,
+// the owners' buffers.  An owner's buffer may be another GPU's memory
+// (NVLink peer addresses).  The kernels use plain loads and stores: no TMA,
+// no multicast.  On one GPU, the owners' buffers are R local allocations, and
+// their concatenation equals the single-GPU receive buffer row for row.
+//
+// The kernels are the simple forms of the single-GPU ones: a warp per
+// (token, 512-channel chunk) for dispatch and the gathers, a warp per pair
+// for combine backward, pieces checked against H one by one.  Peer links
+// (about 0.8 TB/s per direction) rather than HBM bound them.
+#pragma once
+
+#include "movement.cuh"
+
+namespace ep {
+
+constexpr int kMaxPeers = 64;
+
+// Per owner rank: the base of its buffer (row 0 = its first global slot).
+struct PeerRows {
+  void* base[kMaxPeers];
+};
+
+struct PeerParams {
+  int T, H, k, G, chunks;          // T: this rank's tokens
+  int t_begin;                     // global index of this rank's first token
+  int Er;                          // experts per rank
+  const int32_t* slot_of_pair;     // [T_all * k], the global layout
+  const int64_t* topk_idx;         // [T_all * k], every rank's expert ids
+  const int32_t* expert_offset;    // [E + 1], global
+  const float* topk_weights;       // [T * k], this rank's tokens
+};
+
+// Slot, owner rank and the owner's local row of this rank's pair (t, j);
+// slot -1 (masked pair): owner 0, row -1.
+__device__ __forceinline__ int peer_pair(const PeerParams& p, int t, int j, int& owner, int& row) {
+  const int64_t ug = (static_cast<int64_t>(p.t_begin) + t) * p.k + j;
+  const int s = p.slot_of_pair[ug];
+  owner = 0;
+  row = -1;
+  if (s >= 0) {
+    owner = static_cast<int>(p.topk_idx[ug] / p.Er);
+    row = s - p.expert_offset[owner * p.Er];
+  }
+  return s;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kMoveThreads)
+dispatch_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx, PeerRows rscale, PeerRows rweight) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
+       u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
+    const int t = static_cast<int>(u / p.chunks);
+    const int c = static_cast<int>(u - static_cast<int64_t>(t) * p.chunks);
+    const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
+    const bool a0 = h0 < p.H, a1 = h1 < p.H;
+    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    if (a0) v0 = ld_ro_v4(xr + h0);
+    if (a1) v1 = ld_ro_v4(xr + h1);
+    int my_slot = -1, my_owner = 0, my_row = -1;
+    if (lane < p.k) my_slot = peer_pair(p, t, lane, my_owner, my_row);
+    uint2 q0 = make_uint2(0, 0), q1 = q0;
+    float sc0 = 1.0f, sc1 = 1.0f;
+    if constexpr (FP8) {
+      q0 = quantize_piece(v0, sc0);
+      q1 = quantize_piece(v1, sc1);
+    }
+    const bool scale_lane = (lane & (kLanesPerGroup - 1)) == 0;
+    for (int j = 0; j < p.k; ++j) {
+      const int s = __shfl_sync(0xffffffffu, my_slot, j);
+      const int o = __shfl_sync(0xffffffffu, my_owner, j);
+      const int row = __shfl_sync(0xffffffffu, my_row, j);
+      if (s < 0) continue;
+      if constexpr (FP8) {
+        uint8_t* dst = static_cast<uint8_t*>(rx.base[o]) + static_cast<int64_t>(row) * p.H;
+        float* srow = static_cast<float*>(rscale.base[o]) + static_cast<int64_t>(row) * p.G;
+        if (a0) {
+          *reinterpret_cast<uint2*>(dst + h0) = q0;
+          if (scale_lane) srow[h0 / kGroup] = sc0;
+        }
+        if (a1) {
+          *reinterpret_cast<uint2*>(dst + h1) = q1;
+          if (scale_lane) srow[h1 / kGroup] = sc1;
+        }
+      } else {
+        uint16_t* dst = static_cast<uint16_t*>(rx.base[o]) + static_cast<int64_t>(row) * p.H;
+        if (a0) st_v4(dst + h0, v0);
+        if (a1) st_v4(dst + h1, v1);
+      }
+    }
+    if (c == 0 && lane < p.k && my_slot >= 0 && rweight.base[my_owner] != nullptr)
+      static_cast<float*>(rweight.base[my_owner])[my_row] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
+  }
+}
+
+// out[t] = bf16( chain over j of (WEIGHTED ? fmaf(w[t,j], y[slot], acc) : acc + y[slot]) ), acc = +0.0f,
+// j = 0..k-1 in order: the single-GPU arithmetic, rows loaded from their owners.
+template <bool WEIGHTED>
+__global__ void __launch_bounds__(kMoveThreads)
+gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
+       u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
+    const int t = static_cast<int>(u / p.chunks);
+    const int c = static_cast<int>(u - static_cast<int64_t>(t) * p.chunks);
+    const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
+    const bool a0 = h0 < p.H, a1 = h1 < p.H;
+    int my_slot = -1, my_owner = 0, my_row = -1;
+    float my_w = 0.0f;
+    if (lane < p.k) {
+      my_slot = peer_pair(p, t, lane, my_owner, my_row);
+      if (WEIGHTED) my_w = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
+    }
+    float acc[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+    for (int jb = 0; jb < p.k; jb += 8) {  // all loads of a batch of 8 rows in flight, then the arithmetic
+      uint4 v[8][2];
+      int s[8];
+      float w[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const int j = (jb + jj) & (kWarp - 1);
+        s[jj] = __shfl_sync(0xffffffffu, my_slot, j);
+        const int o = __shfl_sync(0xffffffffu, my_owner, j);
+        const int row = __shfl_sync(0xffffffffu, my_row, j);
+        w[jj] = __shfl_sync(0xffffffffu, my_w, j);
+        if (jb + jj >= p.k) s[jj] = -1;
+        v[jj][0] = v[jj][1] = make_uint4(0, 0, 0, 0);
+        if (s[jj] >= 0) {
+          const uint16_t* src = static_cast<const uint16_t*>(y.base[o]) + static_cast<int64_t>(row) * p.H;
+          if (a0) v[jj][0] = *reinterpret_cast<const uint4*>(src + h0);
+          if (a1) v[jj][1] = *reinterpret_cast<const uint4*>(src + h1);
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (s[jj] < 0) continue;
+        float f[16];
+        unpack8(v[jj][0], f);
+        unpack8(v[jj][1], f + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (WEIGHTED) acc[i] = fmaf(w[jj], f[i], acc[i]);
+          else acc[i] = __fadd_rn(acc[i], f[i]);
+        }
+      }
+    }
+    uint16_t* dst = out + static_cast<int64_t>(t) * p.H;
+    if (a0) st_v4(dst + h0, pack8_bf16(acc));
+    if (a1) st_v4(dst + h1, pack8_bf16(acc + 8));
+  }
+}
+
+// grad_y[slot] = bf16(w * g[t]) into the owner's buffer; grad_w[t, j] = g[t] . y[slot] with y from the owner,
+// accumulated per lane in channel order, then across lanes by xor shuffles.
+__global__ void __launch_bounds__(kMoveThreads)
+combine_backward_peers_kernel(PeerParams p, const uint16_t* __restrict__ g, PeerRows y, PeerRows grad_y,
+                              float* __restrict__ grad_w) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int64_t npairs = static_cast<int64_t>(p.T) * p.k;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < npairs;
+       u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
+    const int t = static_cast<int>(u / p.k), j = static_cast<int>(u - static_cast<int64_t>(t) * p.k);
+    int o, row;
+    const int s = peer_pair(p, t, j, o, row);
+    if (s < 0) {
+      if (lane == 0) grad_w[u] = 0.0f;
+      continue;
+    }
+    const float w = p.topk_weights[u];
+    const uint16_t* gr = g + static_cast<int64_t>(t) * p.H;
+    const uint16_t* yr = static_cast<const uint16_t*>(y.base[o]) + static_cast<int64_t>(row) * p.H;
+    uint16_t* dr = static_cast<uint16_t*>(grad_y.base[o]) + static_cast<int64_t>(row) * p.H;
+    float d = 0.0f;
+    for (int c = 0; c < p.chunks; ++c) {
+      const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int hh = h == 0 ? h0 : h1;
+        if (hh >= p.H) continue;
+        const uint4 gv = ld_l1_v4(gr + hh);
+        const uint4 yv = *reinterpret_cast<const uint4*>(yr + hh);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+        uint32_t ov[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
+          d = fmaf(g0, bf16_lo(yw[i]), d);
+          d = fmaf(g1, bf16_hi(yw[i]), d);
+          ov[i] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
+        }
+        st_v4(dr + hh, make_uint4(ov[0], ov[1], ov[2], ov[3]));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (lane == 0) grad_w[u] = d;
+  }
+}
+
+}  // namespace ep

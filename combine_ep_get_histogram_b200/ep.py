@@ -30,7 +30,10 @@ HANDLE_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank"
 EXPORTED = ("ep_handle_sizes", "ep_workspace_size", "ep_get_dispatch_layout", "ep_dispatch",
             "ep_combine", "ep_combine_backward", "ep_dispatch_backward", "ep_get_error",
             "ep_status_string", "ep_last_cuda_error", "ep_get_dispatch_layout_noalloc",
-            "ep_noalloc_scratch_bytes", "ep_route_group_limited")
+            "ep_noalloc_scratch_bytes", "ep_route_group_limited", "ep_dispatch_peers", "ep_combine_peers",
+            "ep_combine_backward_peers", "ep_dispatch_backward_peers")
+
+EP_MAX_PEERS = 64
 
 
 class ep_shape_t(ctypes.Structure):
@@ -40,6 +43,10 @@ class ep_shape_t(ctypes.Structure):
 
 class ep_handle_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in HANDLE_FIELDS]
+
+
+class ep_peer_rows_t(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_void_p * EP_MAX_PEERS)]
 
 
 class EPError(RuntimeError):
@@ -62,6 +69,7 @@ def _lib():
         L = ctypes.CDLL(LIB_PATH)
         vp, i64p = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64)
         shp, hp = ctypes.POINTER(ep_shape_t), ctypes.POINTER(ep_handle_t)
+        pp = ctypes.POINTER(ep_peer_rows_t)
         sig = {
             "ep_handle_sizes": (ctypes.c_int, [shp, i64p]),
             "ep_workspace_size": (ctypes.c_size_t, [shp]),
@@ -76,6 +84,10 @@ def _lib():
             "ep_get_dispatch_layout_noalloc": (ctypes.c_int, [shp, vp, hp, vp]),
             "ep_noalloc_scratch_bytes": (ctypes.c_size_t, []),
             "ep_route_group_limited": (ctypes.c_int, [shp, vp, ctypes.c_int, ctypes.c_int, vp, vp, vp]),
+            "ep_dispatch_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, vp, vp, pp, pp, pp, vp]),
+            "ep_combine_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, pp, vp, vp, vp]),
+            "ep_combine_backward_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, vp, pp, vp, pp, vp, vp]),
+            "ep_dispatch_backward_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, pp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -219,3 +231,56 @@ def ep_route_group_limited(shape: ep_shape_t, scores, n_groups: int, topk_groups
 def ep_get_error(handle: Handle, stream=None) -> int:
     """Synchronises the stream; returns EP_OK or EP_ERR_BAD_INDEX (and clears it)."""
     return _lib().ep_get_error(ctypes.byref(handle.c), _stream(stream))
+
+
+# ---------------------------------------------------- multi-GPU (one rank per GPU)
+
+def peer_rows(buffers) -> ep_peer_rows_t | None:
+    """Peer table for the *_peers calls: buffers[o] is owner rank o's buffer
+    (a tensor or a raw device pointer, possibly another GPU's memory), or
+    None for no table."""
+    if buffers is None:
+        return None
+    if len(buffers) > EP_MAX_PEERS:
+        raise ValueError(f"at most {EP_MAX_PEERS} ranks")
+    t = ep_peer_rows_t()
+    for o, b in enumerate(buffers):
+        t.rows[o] = _ptr(b)
+    return t
+
+
+def _byref(t):
+    return None if t is None else ctypes.byref(t)
+
+
+def ep_dispatch_peers(shape: ep_shape_t, rank: int, topk_idx, handle: Handle, x, topk_weights, recv_x,
+                      recv_scale=None, recv_weight=None, stream=None, check=True) -> int:
+    """This rank's tokens into their owners' receive buffers (recv_*: one
+    buffer per owner rank)."""
+    st = _lib().ep_dispatch_peers(ctypes.byref(shape), rank, _ptr(topk_idx), ctypes.byref(handle.c), _ptr(x),
+                                  _ptr(topk_weights), _byref(peer_rows(recv_x)), _byref(peer_rows(recv_scale)),
+                                  _byref(peer_rows(recv_weight)), _stream(stream))
+    return _check(st, "ep_dispatch_peers") if check else st
+
+
+def ep_combine_peers(shape: ep_shape_t, rank: int, topk_idx, handle: Handle, y, topk_weights, out, stream=None,
+                     check=True) -> int:
+    """This rank's tokens, combined from the owners' expert outputs (y: one buffer per owner rank)."""
+    st = _lib().ep_combine_peers(ctypes.byref(shape), rank, _ptr(topk_idx), ctypes.byref(handle.c),
+                                 _byref(peer_rows(y)), _ptr(topk_weights), _ptr(out), _stream(stream))
+    return _check(st, "ep_combine_peers") if check else st
+
+
+def ep_combine_backward_peers(shape: ep_shape_t, rank: int, topk_idx, handle: Handle, grad_out, y, topk_weights,
+                              grad_y, grad_w, stream=None, check=True) -> int:
+    st = _lib().ep_combine_backward_peers(ctypes.byref(shape), rank, _ptr(topk_idx), ctypes.byref(handle.c),
+                                          _ptr(grad_out), _byref(peer_rows(y)), _ptr(topk_weights),
+                                          _byref(peer_rows(grad_y)), _ptr(grad_w), _stream(stream))
+    return _check(st, "ep_combine_backward_peers") if check else st
+
+
+def ep_dispatch_backward_peers(shape: ep_shape_t, rank: int, topk_idx, handle: Handle, grad_recv, grad_x,
+                               stream=None, check=True) -> int:
+    st = _lib().ep_dispatch_backward_peers(ctypes.byref(shape), rank, _ptr(topk_idx), ctypes.byref(handle.c),
+                                           _byref(peer_rows(grad_recv)), _ptr(grad_x), _stream(stream))
+    return _check(st, "ep_dispatch_backward_peers") if check else st

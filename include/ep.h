@@ -209,6 +209,52 @@ size_t ep_noalloc_scratch_bytes(void);
 int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_groups, int topk_groups,
                            int64_t* topk_idx, float* topk_weights, ep_stream_t stream);
 
+/* ---- Multi-GPU expert parallelism: one process per GPU -----------------
+ *
+ * R ranks, one GPU each (the pages' EP8 over NVLink: blog.hotdry.top
+ * "deepep-expert-parallel-communication-library", section 一; dispatch and
+ * combine are all-to-alls between ranks: zhouruolin.cn, section 五).  Rank r
+ * holds tokens [r*T/R, (r+1)*T/R) and experts [r*E/R, (r+1)*E/R).  Every
+ * rank gathers all ranks' topk_idx ([T,k], T*k*8 bytes) and runs
+ * ep_get_dispatch_layout over it, so every rank holds the same global
+ * layout.  Owner rank o keeps the global receive rows
+ * [expert_offset[o*E/R], expert_offset[(o+1)*E/R]) in its own buffers, row
+ * expert_offset[o*E/R] first; the concatenation over o of those buffers is
+ * the single-GPU receive buffer.  The calls below move this rank's tokens
+ * only, and read or write each receive row in its owner's buffer, which may
+ * be another GPU's memory (a peer address reachable from this device: CUDA
+ * IPC, or memory allocated for symmetric access).  Loads and stores are
+ * plain ones, with no TMA and no multicast.  The arithmetic is that of the
+ * single-GPU calls, element for element.
+ *
+ * shape: the global problem (T = all ranks' tokens); R <= EP_MAX_PEERS.
+ * rank: this process's rank.  topk_idx: [T,k] int64, every rank's ids (the
+ * layout's input).  handle: the global layout.  Per-rank arrays (x,
+ * topk_weights, out, grad_out, grad_w, grad_x) hold this rank's T/R tokens.
+ * Peer tables give, for every owner o < R, the base of o's buffer: rows of
+ * H bf16 (or H E4M3 bytes for recv_x under FP8), H/128 fp32 scales, or one
+ * fp32 weight per row; 16-byte aligned.  recv_weight may be NULL (no
+ * weights written).  Same stream ordering, no allocation and no sync as the
+ * single-GPU calls; the caller orders the ranks' calls (a barrier or
+ * events between a buffer's writers and its readers). */
+#define EP_MAX_PEERS 64
+typedef struct {
+  void* rows[EP_MAX_PEERS];
+} ep_peer_rows_t;
+
+int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, const ep_handle_t* handle,
+                      const void* x, const float* topk_weights, const ep_peer_rows_t* recv_x,
+                      const ep_peer_rows_t* recv_scale, const ep_peer_rows_t* recv_weight, ep_stream_t stream);
+int ep_combine_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, const ep_handle_t* handle,
+                     const ep_peer_rows_t* y, const float* topk_weights, void* out, ep_stream_t stream);
+int ep_combine_backward_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx,
+                              const ep_handle_t* handle, const void* grad_out, const ep_peer_rows_t* y,
+                              const float* topk_weights, const ep_peer_rows_t* grad_y, float* grad_w,
+                              ep_stream_t stream);
+int ep_dispatch_backward_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx,
+                               const ep_handle_t* handle, const ep_peer_rows_t* grad_recv, void* grad_x,
+                               ep_stream_t stream);
+
 /* Synchronises `stream`, reads handle->error_word, clears it, and returns
  * EP_ERR_BAD_INDEX if a bad expert id was seen since the last read, else
  * EP_ERR_CAPACITY if a padded block overflowed, else EP_OK; EP_ERR_CUDA if

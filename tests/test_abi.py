@@ -107,6 +107,39 @@ def test_bad_pointers_rejected_on_host():
     assert lib.ep_get_error(None, None) == 1
 
 
+def test_peer_calls_reject_bad_arguments_on_host():
+    """The multi-GPU calls check rank, shape and every owner's buffer before
+    any device work (no GPU needed to see the rejections)."""
+    s = ep.make_shape(T=64, H=256, k=4, E=16, R=4, use_fp8=True)
+    lib = ep.library()
+    good = 1 << 20
+    h = binding.ep_handle_t(*([good] * 9))
+    sref, href = ctypes.byref(s), ctypes.byref(h)
+    rows = binding.peer_rows([good] * 4)
+    one_short = binding.peer_rows([good] * 3)            # owner 3 missing
+    odd = binding.peer_rows([good, good + 8, good, good])  # owner 1 not 16-byte aligned
+    rr = ctypes.byref(rows)
+    # rank out of range, null / misaligned topk_idx, null weights
+    assert lib.ep_dispatch_peers(sref, 4, good, href, good, good, rr, rr, None, None) == 1
+    assert lib.ep_dispatch_peers(sref, -1, good, href, good, good, rr, rr, None, None) == 1
+    assert lib.ep_dispatch_peers(sref, 0, None, href, good, good, rr, rr, None, None) == 1
+    assert lib.ep_dispatch_peers(sref, 0, good + 4, href, good, good, rr, rr, None, None) == 1
+    assert lib.ep_dispatch_peers(sref, 0, good, href, good, None, rr, rr, None, None) == 1
+    # every owner's buffer present and aligned; FP8 needs the scale table
+    assert lib.ep_dispatch_peers(sref, 0, good, href, good, good, ctypes.byref(one_short), rr, None, None) == 1
+    assert lib.ep_dispatch_peers(sref, 0, good, href, good, good, ctypes.byref(odd), rr, None, None) == 1
+    assert lib.ep_dispatch_peers(sref, 0, good, href, good, good, rr, None, None, None) == 1
+    assert lib.ep_combine_peers(sref, 0, good, href, None, good, good, None) == 1
+    assert lib.ep_combine_peers(sref, 0, good, href, ctypes.byref(odd), good, good, None) == 1
+    assert lib.ep_combine_backward_peers(sref, 0, good, href, good, rr, good, None, good, None) == 1
+    assert lib.ep_dispatch_backward_peers(sref, 0, good, href, rr, good + 2, None) == 1
+    # more ranks than the peer table holds; the padded layout has no peer form
+    big = ep.make_shape(T=128, H=256, k=4, E=128, R=128)
+    assert lib.ep_combine_peers(ctypes.byref(big), 0, good, href, rr, good, good, None) == 1
+    padded = ep.make_shape(T=64, H=256, k=4, E=16, R=4, max_tokens_per_rank=16)
+    assert lib.ep_combine_peers(ctypes.byref(padded), 0, good, href, rr, good, good, None) == 1
+
+
 def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(binding, "_LIB", None)
