@@ -537,6 +537,7 @@ def run_ours(args, rank, world, local):
         del paths[1]
 
     overlap = measure_overlap(args, w, d, dev, M, ms_per_step) if args.overlap_sms else None
+    load = load_skew(path.handle, w)
 
     if rank != 0:
         return None
@@ -579,9 +580,28 @@ def run_ours(args, rank, world, local):
         "timing": "CUDA graph replay of the step" if not args.no_graph else "eager launches",
         "e2e": e2e,
     }
+    line["load"] = load
     if overlap is not None:
         line["overlap"] = overlap
     return line
+
+
+def load_skew(handle, w) -> dict:
+    """Load balance of the step's routing from the layout's counts (read
+    after the timed region): the busiest expert's and the busiest rank's
+    receive counts over their means.  The pages use max > 2x mean as the sign
+    of skew."""
+    per_expert = handle.tensors["num_tokens_per_expert"].cpu().numpy().astype(float)
+    per_rank = handle.tensors["num_tokens_per_rank"].cpu().numpy().astype(float)
+    er = w.E // w.R
+    rows_per_rank = per_expert.reshape(w.R, er).sum(axis=1)
+
+    def ratio(v):
+        return round(float(v.max() / v.mean()), 3) if v.size and v.mean() > 0 else None
+
+    return {"tokens_per_expert_max_over_mean": ratio(per_expert),
+            "rows_per_rank_max_over_mean": ratio(rows_per_rank),
+            "tokens_per_rank_max_over_mean": ratio(per_rank)}
 
 
 def measure_overlap(args, w, d, dev, M, step_ms):

@@ -44,3 +44,18 @@ def test_l2_statement_follows_the_step_bytes():
     assert not flush and "no flush" in text
     flush, text = bench.l2_policy(4 * l2 - 1, l2)
     assert flush and "flushed" in text
+
+
+def test_load_skew_is_max_over_mean_of_the_layout_counts():
+    import torch
+    from combine_ep_get_histogram_b200 import workloads as wl
+
+    class FakeHandle:
+        tensors = {"num_tokens_per_expert": torch.tensor([6, 2, 2, 2, 1, 1, 1, 1], dtype=torch.int32),
+                   "num_tokens_per_rank": torch.tensor([5, 3], dtype=torch.int32)}
+
+    w = wl.Workload("t", T=8, H=128, k=2, E=8, R=2, use_fp8=False, routing="group")
+    load = bench.load_skew(FakeHandle(), w)
+    assert load["tokens_per_expert_max_over_mean"] == 6 / 2
+    assert load["rows_per_rank_max_over_mean"] == round(12 / 8, 3)  # rank rows 12 and 4
+    assert load["tokens_per_rank_max_over_mean"] == round(5 / 4, 3)
