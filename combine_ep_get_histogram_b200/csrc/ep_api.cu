@@ -1,6 +1,8 @@
 // C ABI of libep_b200.so (declared in include/ep.h): argument checks on the
-// host, launch configuration, status codes.  Every step of the hot path runs
-// in the kernels of layout.cuh and movement.cuh; nothing here touches data.
+// host, launch configuration, status codes.  Every step runs in the kernels of
+// layout.cuh (routing layout), movement.cuh (dispatch, combine, backward
+// passes), route.cuh (group-limited routing) and peers.cuh (the multi-GPU
+// forms); nothing here touches data.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -74,7 +76,9 @@ int device_info(const DeviceInfo** out) {
     d.sms = prop.multiProcessorCount;
     d.supported = prop.major == 10 && prop.minor == 0;
     if (d.supported) {
-      cudaFuncSetAttribute(reinterpret_cast<const void*>(layout_padded_kernel),
+      cudaFuncSetAttribute(reinterpret_cast<const void*>(layout_padded_kernel<true>),
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, kPadMaxSmem);
+      cudaFuncSetAttribute(reinterpret_cast<const void*>(layout_padded_kernel<false>),
                            cudaFuncAttributeMaxDynamicSharedMemorySize, kPadMaxSmem);
       d.occ_count = occupancy(reinterpret_cast<const void*>(layout_count_kernel), kLayoutThreads,
                               (kMaxE + kMaxR) * 4 + kTileFlagBytes);
@@ -311,11 +315,29 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (shape->max_tokens_per_rank > 0) {
+    const size_t smem = layout_padded_smem(p.Tr, shape->E, shape->R);
+    if (shape->R <= kPadClusterMax) {  // one cluster of R CTAs sums the totals itself
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(shape->R);
+      cfg.blockDim = dim3(kPadThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = shape->R;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if ((st = cuda_status(cudaLaunchKernelEx(&cfg, layout_padded_kernel<true>, p, shape->max_tokens_per_rank))) !=
+          EP_OK)
+        return st;
+      return finish(handle, s);
+    }
     if ((st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_expert, 0, shape->E * 4, s))) != EP_OK ||
         (st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_rank, 0, shape->R * 4, s))) != EP_OK)
       return st;
-    layout_padded_kernel<<<shape->R, kPadThreads, layout_padded_smem(p.Tr, shape->E, shape->R), s>>>(
-        p, shape->max_tokens_per_rank);
+    layout_padded_kernel<false><<<shape->R, kPadThreads, smem, s>>>(p, shape->max_tokens_per_rank);
     return finish(handle, s);
   }
   if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {

@@ -471,21 +471,27 @@ layout_small_kernel(LayoutParams p) {
 // launch: per-warp expert histograms of the rank's pairs (contiguous runs),
 // an exclusive scan over warps per expert from 0, ranking with
 // popc(same_expert_mask & lanemask_lt).  Totals over ranks
-// (num_tokens_per_expert, num_tokens_per_rank) are integer atomics into
-// arrays zeroed just before the launch, so their values do not depend on
-// order.  Rows a block does not fill are marked -1 in src_of_slot.
+// (num_tokens_per_expert, num_tokens_per_rank): with R <= kPadClusterMax the
+// R CTAs are one thread-block cluster, and after a cluster barrier CTA c sums
+// its slice of the experts and ranks over every CTA's counts through
+// distributed shared memory (no atomics, nothing to zero first); with more
+// ranks they are integer atomics into arrays zeroed just before the launch.
+// Either way the values do not depend on order.  Rows a block does not fill
+// are marked -1 in src_of_slot.
 
 constexpr int kPadThreads = 512;
 constexpr int kPadWarps = kPadThreads / kWarp;
 constexpr int kPadMaxPairs = 8192;   // pairs of one source rank
 constexpr int kPadMaxFlags = 32768;  // (T/R) x R token-rank flag bytes
 constexpr int kPadChunks = (kPadMaxPairs / kPadWarps + kWarp - 1) / kWarp;  // 16
+constexpr int kPadClusterMax = 8;    // portable cluster size
 
 __host__ __device__ inline int layout_padded_smem(int Tr, int E, int R) {
   return (kPadWarps * E + E + R) * 4 + Tr * R;  // whist[W][E] cnt[E] rank_cnt[R] flags[Tr][R]
 }
 constexpr int kPadMaxSmem = (kPadWarps * kMaxE + kMaxE + kMaxR) * 4 + kPadMaxFlags;
 
+template <bool CLUSTER>
 __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams p, int M) {
   extern __shared__ int32_t smem[];
   int32_t* whist = smem;                         // [W][E]
@@ -533,7 +539,7 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
     cnt[e] = run;
     p.count_src_rank_expert[r * p.E + e] = run;
     p.src_rank_expert_offset[r * p.E + e] = (e * p.R + r) * M;
-    if (run > 0) atomicAdd(&p.num_tokens_per_expert[e], run);
+    if (!CLUSTER && run > 0) atomicAdd(&p.num_tokens_per_expert[e], run);
   }
   if (r == 0)
     for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.expert_offset[e] = e * p.R * M;
@@ -579,8 +585,28 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
     if (key >= 0 && lane == __ffs(same) - 1) atomicAdd(&rank_cnt[key], __popc(same));
   }
   __syncthreads();
-  for (int d = threadIdx.x; d < p.R; d += blockDim.x)
-    if (rank_cnt[d] > 0) atomicAdd(&p.num_tokens_per_rank[d], rank_cnt[d]);
+  if constexpr (CLUSTER) {
+    // every CTA's cnt and rank_cnt are final; CTA r sums its slice of the
+    // experts and of the destination ranks over the cluster
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int e_lo = r * p.E / p.R, e_hi = (r + 1) * p.E / p.R;
+    for (int e = e_lo + threadIdx.x; e < e_hi; e += blockDim.x) {
+      int32_t n = 0;
+      for (int q = 0; q < p.R; ++q) n += cluster.map_shared_rank(cnt, q)[e];
+      p.num_tokens_per_expert[e] = n;
+    }
+    if (threadIdx.x == 0) {
+      int32_t n = 0;
+      for (int q = 0; q < p.R; ++q) n += cluster.map_shared_rank(rank_cnt, q)[r];
+      p.num_tokens_per_rank[r] = n;
+    }
+    cluster.sync();  // keep this CTA's shared memory until the others have read it
+  } else {
+    for (int d = threadIdx.x; d < p.R; d += blockDim.x)
+      if (rank_cnt[d] > 0) atomicAdd(&p.num_tokens_per_rank[d], rank_cnt[d]);
+  }
   if (bad) atomicOr(p.error_word, 1);
   if (over) atomicOr(p.error_word, 2);
 }

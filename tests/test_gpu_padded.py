@@ -77,6 +77,15 @@ def test_padded_low_latency_shape(cuda_device, M, use_fp8):
     run_padded(cuda_device, T, H, k, E, R, M, use_fp8, routing(T, k, E, seed=M))
 
 
+@pytest.mark.parametrize("R", [1, 3, 16, 32])
+def test_padded_rank_counts(cuda_device, R):
+    """Up to 8 ranks the layout is one cluster of R CTAs that sums the totals
+    through distributed shared memory (R = 1 and an odd R = 3 included);
+    past 8 the totals are atomics into zeroed arrays."""
+    T, H, k, E = 384, 256, 4, 96
+    run_padded(cuda_device, T, H, k, E, R, T // R + 2, R % 2 == 1, routing(T, k, E, seed=R, masked=0.1))
+
+
 def test_padded_capacity_overflow_masked_and_bad(cuda_device):
     T, H, k, E, R = 64, 256, 4, 8, 4
     idx = routing(T, k, E, seed=3, masked=0.2, duplicates=True)
