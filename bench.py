@@ -299,7 +299,14 @@ class PeersPath(Path):
         self.ranks = [(r, slice(r * Tl, (r + 1) * Tl)) for r in range(w.R)]
 
     def step(self, marks=None, before_back=None, after_combine=None):
+        """One step; every call runs its R ranks on R streams forked from and
+        joined back to the current stream, as the ranks of R GPUs would run
+        side by side."""
+        import torch
         ep, i, sh, h = self.ep, self.inp, self.shape, self.handle
+        cur = torch.cuda.current_stream()
+        if not hasattr(self, "rank_streams"):
+            self.rank_streams = [torch.cuda.Stream(self.dev) for _ in self.ranks]
         n = 0
 
         def rec():
@@ -308,26 +315,34 @@ class PeersPath(Path):
                 marks[n].record()
             n += 1
 
+        def fanout(call):
+            fork = torch.cuda.Event()
+            fork.record(cur)
+            for (r, tok), st in zip(self.ranks, self.rank_streams):
+                st.wait_event(fork)
+                with torch.cuda.stream(st):
+                    call(r, tok)
+                done = torch.cuda.Event()
+                done.record(st)
+                cur.wait_event(done)
+
         rec()
         ep.ep_get_dispatch_layout(sh, i["topk_idx"], h, self.ws)
         rec()
-        for r, tok in self.ranks:
-            ep.ep_dispatch_peers(sh, r, i["topk_idx"], h, i["x"][tok], i["topk_weights"][tok], self.rx, self.rs,
-                                 self.rw)
+        fanout(lambda r, tok: ep.ep_dispatch_peers(sh, r, i["topk_idx"], h, i["x"][tok], i["topk_weights"][tok],
+                                                   self.rx, self.rs, self.rw))
         rec()
         if before_back is not None:
             before_back()
-        for r, tok in self.ranks:
-            ep.ep_combine_peers(sh, r, i["topk_idx"], h, self.ys, i["topk_weights"][tok], self.out[tok])
+        fanout(lambda r, tok: ep.ep_combine_peers(sh, r, i["topk_idx"], h, self.ys, i["topk_weights"][tok],
+                                                  self.out[tok]))
         if after_combine is not None:
             after_combine()
         rec()
-        for r, tok in self.ranks:
-            ep.ep_combine_backward_peers(sh, r, i["topk_idx"], h, i["g"][tok], self.ys, i["topk_weights"][tok],
-                                         self.gy, self.grad_w[tok])
+        fanout(lambda r, tok: ep.ep_combine_backward_peers(sh, r, i["topk_idx"], h, i["g"][tok], self.ys,
+                                                           i["topk_weights"][tok], self.gy, self.grad_w[tok]))
         rec()
-        for r, tok in self.ranks:
-            ep.ep_dispatch_backward_peers(sh, r, i["topk_idx"], h, self.gy, self.grad_x[tok])
+        fanout(lambda r, tok: ep.ep_dispatch_backward_peers(sh, r, i["topk_idx"], h, self.gy, self.grad_x[tok]))
         rec()
 
 
@@ -553,8 +568,14 @@ def run_ours(args, rank, world, local):
     kernel_of = {"dispatch": "dispatch_tma_kernel<FP8>" if w.use_fp8 else "dispatch_tma_kernel<BF16>",
                  "combine": "gather_reduce_kernel<weighted>", "combine_backward": "combine_backward_kernel",
                  "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel",
-                 "route": "route_group_limited_kernel"}
+                 "route": "route_aligned_kernel|route_group_limited_kernel"}
+    if args.peers:
+        kernel_of.update({"dispatch": "dispatch_peers_kernel", "combine": "gather_reduce_peers_kernel<weighted>",
+                          "combine_backward": "combine_backward_peers_kernel",
+                          "dispatch_backward": "gather_reduce_peers_kernel<unweighted>"})
     ach = per_call[dominant]["GB_s"]
+    # the stored capture is of the single-GPU kernel; the peer kernels have none
+    traffic = None if args.peers else measured_traffic(w, dominant)
     line = {
         "metric": METRIC,
         "value": round(job_gbs(step_bytes, args.steps, world, total_ms), 2),
@@ -573,7 +594,7 @@ def run_ours(args, rank, world, local):
         "roofline": {"kernel": kernel_of[dominant], "call": dominant, "bound": "hbm", "achieved": ach,
                      "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 3),
                      "peak_source": f"{peak_kind} hbm_gbs",
-                     "bytes_per_launch": nb[dominant], "traffic": measured_traffic(w, dominant),
+                     "bytes_per_launch": nb[dominant], "traffic": traffic,
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, full-size launch"},
         "clocks": clocks,
         "gpu_launches": (launches_per_step(w, args.peers) + (1 if args.route else 0)) * args.steps,

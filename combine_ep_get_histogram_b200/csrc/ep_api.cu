@@ -46,7 +46,7 @@ struct DeviceInfo {
   int occ_comb[2] = {}, occ_dbwd[2] = {};  // [ragged]
   int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
   int occ_cbwd[2] = {};  // [ragged]
-  int occ_peer_disp[2] = {}, occ_peer_gather[2] = {}, occ_peer_cbwd = 0;  // [fp8], [weighted]
+  int occ_peer_disp[2] = {}, occ_peer_gather[2][2] = {}, occ_peer_cbwd[2] = {};  // [fp8], [weighted][ragged], [ragged]
   int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
   int occ_route_aligned[6] = {};  // route_aligned_kernel<1, 2, 4, 8, 16, 32>
 };
@@ -92,11 +92,18 @@ int device_info(const DeviceInfo** out) {
       d.occ_cbwd[1] = occupancy(reinterpret_cast<const void*>(combine_backward_kernel<true>), kMoveThreads, 0);
       d.occ_peer_disp[0] = occupancy(reinterpret_cast<const void*>(dispatch_peers_kernel<false>), kMoveThreads, 0);
       d.occ_peer_disp[1] = occupancy(reinterpret_cast<const void*>(dispatch_peers_kernel<true>), kMoveThreads, 0);
-      d.occ_peer_gather[0] =
-          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<false>), kMoveThreads, 0);
-      d.occ_peer_gather[1] =
-          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<true>), kMoveThreads, 0);
-      d.occ_peer_cbwd = occupancy(reinterpret_cast<const void*>(combine_backward_peers_kernel), kMoveThreads, 0);
+      d.occ_peer_gather[0][0] =
+          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<false, false>), kMoveThreads, 0);
+      d.occ_peer_gather[0][1] =
+          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<false, true>), kMoveThreads, 0);
+      d.occ_peer_gather[1][0] =
+          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<true, false>), kMoveThreads, 0);
+      d.occ_peer_gather[1][1] =
+          occupancy(reinterpret_cast<const void*>(gather_reduce_peers_kernel<true, true>), kMoveThreads, 0);
+      d.occ_peer_cbwd[0] =
+          occupancy(reinterpret_cast<const void*>(combine_backward_peers_kernel<false>), kMoveThreads, 0);
+      d.occ_peer_cbwd[1] =
+          occupancy(reinterpret_cast<const void*>(combine_backward_peers_kernel<true>), kMoveThreads, 0);
       const void* route_fns[6] = {reinterpret_cast<const void*>(route_group_limited_kernel<1>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<2>),
                                   reinterpret_cast<const void*>(route_group_limited_kernel<4>),
@@ -252,6 +259,7 @@ int peer_setup(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, c
   p->chunks = static_cast<int>(ceil_div(shape->H, kChunk));
   p->t_begin = static_cast<int>(rank * Tl);
   p->Er = shape->E / shape->R;
+  p->R = shape->R;
   p->slot_of_pair = handle->slot_of_pair;
   p->topk_idx = topk_idx;
   p->expert_offset = handle->expert_offset;
@@ -562,8 +570,13 @@ int ep_combine_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_
   if ((st = device_info(&d)) != EP_OK) return st;
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int grid = movement_grid(*d, shape, d->occ_peer_gather[1], static_cast<int64_t>(p.T) * p.chunks);
-  gather_reduce_peers_kernel<true><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(y), static_cast<uint16_t*>(out));
+  const bool ragged = shape->H % kChunk != 0;
+  const int grid = movement_grid(*d, shape, d->occ_peer_gather[1][ragged], static_cast<int64_t>(p.T) * p.chunks);
+  if (ragged)
+    gather_reduce_peers_kernel<true, true><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(y), static_cast<uint16_t*>(out));
+  else
+    gather_reduce_peers_kernel<true, false><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(y),
+                                                                         static_cast<uint16_t*>(out));
   return finish(handle, s);
 }
 
@@ -583,9 +596,14 @@ int ep_combine_backward_peers(const ep_shape_t* shape, int32_t rank, const int64
   if ((st = device_info(&d)) != EP_OK) return st;
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int grid = movement_grid(*d, shape, d->occ_peer_cbwd, static_cast<int64_t>(p.T) * p.k);
-  combine_backward_peers_kernel<<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_out),
-                                                             peer_rows(y), peer_rows(grad_y), grad_w);
+  const bool ragged = shape->H % kChunk != 0;
+  const int grid = movement_grid(*d, shape, d->occ_peer_cbwd[ragged], static_cast<int64_t>(p.T) * p.k);
+  const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
+  if (ragged)
+    combine_backward_peers_kernel<true><<<grid, kMoveThreads, 0, s>>>(p, gp, peer_rows(y), peer_rows(grad_y), grad_w);
+  else
+    combine_backward_peers_kernel<false><<<grid, kMoveThreads, 0, s>>>(p, gp, peer_rows(y), peer_rows(grad_y),
+                                                                      grad_w);
   return finish(handle, s);
 }
 
@@ -600,9 +618,14 @@ int ep_dispatch_backward_peers(const ep_shape_t* shape, int32_t rank, const int6
   if ((st = device_info(&d)) != EP_OK) return st;
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int grid = movement_grid(*d, shape, d->occ_peer_gather[0], static_cast<int64_t>(p.T) * p.chunks);
-  gather_reduce_peers_kernel<false><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(grad_recv),
-                                                                 static_cast<uint16_t*>(grad_x));
+  const bool ragged = shape->H % kChunk != 0;
+  const int grid = movement_grid(*d, shape, d->occ_peer_gather[0][ragged], static_cast<int64_t>(p.T) * p.chunks);
+  if (ragged)
+    gather_reduce_peers_kernel<false, true><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(grad_recv),
+                                                                         static_cast<uint16_t*>(grad_x));
+  else
+    gather_reduce_peers_kernel<false, false><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(grad_recv),
+                                                                          static_cast<uint16_t*>(grad_x));
   return finish(handle, s);
 }
 

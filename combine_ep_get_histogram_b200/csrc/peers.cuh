@@ -18,10 +18,12 @@
 // no multicast.  On one GPU, the owners' buffers are R local allocations, and
 // their concatenation equals the single-GPU receive buffer row for row.
 //
-// The kernels are the simple forms of the single-GPU ones: a warp per
-// (token, 512-channel chunk) for dispatch and the gathers, a warp per pair
-// for combine backward, pieces checked against H one by one.  Peer links
-// (about 0.8 TB/s per direction) rather than HBM bound them.
+// The kernels follow the single-GPU ones: a warp per (token, 512-channel
+// chunk) for dispatch and the gathers (their k row loads in flight in
+// batches of 8), a warp per pair for combine backward (four chunks at a time,
+// one partial sum each), bounds checked per piece only when H is not a
+// multiple of 512.  Dispatch stores 16-byte pieces rather than TMA rows.
+// Peer links (about 0.8 TB/s per direction) rather than HBM bound them.
 #pragma once
 
 #include "movement.cuh"
@@ -38,23 +40,32 @@ struct PeerRows {
 struct PeerParams {
   int T, H, k, G, chunks;          // T: this rank's tokens
   int t_begin;                     // global index of this rank's first token
-  int Er;                          // experts per rank
+  int Er, R;                       // experts per rank, ranks
   const int32_t* slot_of_pair;     // [T_all * k], the global layout
   const int64_t* topk_idx;         // [T_all * k], every rank's expert ids
   const int32_t* expert_offset;    // [E + 1], global
   const float* topk_weights;       // [T * k], this rank's tokens
 };
 
+// Every owner's first global row, staged in shared memory once per CTA so
+// that a pair's local row needs no dependent global load.
+__device__ __forceinline__ void load_owner_rows(const PeerParams& p, int32_t* row0) {
+  for (int o = threadIdx.x; o < p.R; o += blockDim.x) row0[o] = p.expert_offset[o * p.Er];
+  __syncthreads();
+}
+
 // Slot, owner rank and the owner's local row of this rank's pair (t, j);
 // slot -1 (masked pair): owner 0, row -1.
-__device__ __forceinline__ int peer_pair(const PeerParams& p, int t, int j, int& owner, int& row) {
+__device__ __forceinline__ int peer_pair(const PeerParams& p, const int32_t* row0, int t, int j, int& owner,
+                                         int& row) {
   const int64_t ug = (static_cast<int64_t>(p.t_begin) + t) * p.k + j;
   const int s = p.slot_of_pair[ug];
+  const int64_t e = p.topk_idx[ug];
   owner = 0;
   row = -1;
   if (s >= 0) {
-    owner = static_cast<int>(p.topk_idx[ug] / p.Er);
-    row = s - p.expert_offset[owner * p.Er];
+    owner = static_cast<int>(e / p.Er);
+    row = s - row0[owner];
   }
   return s;
 }
@@ -62,6 +73,8 @@ __device__ __forceinline__ int peer_pair(const PeerParams& p, int t, int j, int&
 template <bool FP8>
 __global__ void __launch_bounds__(kMoveThreads)
 dispatch_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx, PeerRows rscale, PeerRows rweight) {
+  __shared__ int32_t row0[kMaxPeers];
+  load_owner_rows(p, row0);
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
@@ -75,7 +88,7 @@ dispatch_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx,
     if (a0) v0 = ld_ro_v4(xr + h0);
     if (a1) v1 = ld_ro_v4(xr + h1);
     int my_slot = -1, my_owner = 0, my_row = -1;
-    if (lane < p.k) my_slot = peer_pair(p, t, lane, my_owner, my_row);
+    if (lane < p.k) my_slot = peer_pair(p, row0, t, lane, my_owner, my_row);
     uint2 q0 = make_uint2(0, 0), q1 = q0;
     float sc0 = 1.0f, sc1 = 1.0f;
     if constexpr (FP8) {
@@ -112,9 +125,11 @@ dispatch_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx,
 
 // out[t] = bf16( chain over j of (WEIGHTED ? fmaf(w[t,j], y[slot], acc) : acc + y[slot]) ), acc = +0.0f,
 // j = 0..k-1 in order: the single-GPU arithmetic, rows loaded from their owners.
-template <bool WEIGHTED>
+template <bool WEIGHTED, bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out) {
+  __shared__ int32_t row0[kMaxPeers];
+  load_owner_rows(p, row0);
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
@@ -122,11 +137,11 @@ gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out)
     const int t = static_cast<int>(u / p.chunks);
     const int c = static_cast<int>(u - static_cast<int64_t>(t) * p.chunks);
     const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
-    const bool a0 = h0 < p.H, a1 = h1 < p.H;
+    const bool a0 = !RAGGED || h0 < p.H, a1 = !RAGGED || h1 < p.H;
     int my_slot = -1, my_owner = 0, my_row = -1;
     float my_w = 0.0f;
     if (lane < p.k) {
-      my_slot = peer_pair(p, t, lane, my_owner, my_row);
+      my_slot = peer_pair(p, row0, t, lane, my_owner, my_row);
       if (WEIGHTED) my_w = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
     }
     float acc[16];
@@ -170,18 +185,22 @@ gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out)
   }
 }
 
-// grad_y[slot] = bf16(w * g[t]) into the owner's buffer; grad_w[t, j] = g[t] . y[slot] with y from the owner,
-// accumulated per lane in channel order, then across lanes by xor shuffles.
+// grad_y[slot] = bf16(w * g[t]) into the owner's buffer; grad_w[t, j] = g[t] . y[slot] with y from the owner:
+// four chunks at a time with one fp32 partial sum per chunk slot, then xor shuffles across lanes (the
+// single-GPU kernel's order).
+template <bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 combine_backward_peers_kernel(PeerParams p, const uint16_t* __restrict__ g, PeerRows y, PeerRows grad_y,
                               float* __restrict__ grad_w) {
+  __shared__ int32_t row0[kMaxPeers];
+  load_owner_rows(p, row0);
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t npairs = static_cast<int64_t>(p.T) * p.k;
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < npairs;
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int t = static_cast<int>(u / p.k), j = static_cast<int>(u - static_cast<int64_t>(t) * p.k);
     int o, row;
-    const int s = peer_pair(p, t, j, o, row);
+    const int s = peer_pair(p, row0, t, j, o, row);
     if (s < 0) {
       if (lane == 0) grad_w[u] = 0.0f;
       continue;
@@ -190,31 +209,54 @@ combine_backward_peers_kernel(PeerParams p, const uint16_t* __restrict__ g, Peer
     const uint16_t* gr = g + static_cast<int64_t>(t) * p.H;
     const uint16_t* yr = static_cast<const uint16_t*>(y.base[o]) + static_cast<int64_t>(row) * p.H;
     uint16_t* dr = static_cast<uint16_t*>(grad_y.base[o]) + static_cast<int64_t>(row) * p.H;
-    float d = 0.0f;
-    for (int c = 0; c < p.chunks; ++c) {
-      const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
+    float d[kCbwdUnroll];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int hh = h == 0 ? h0 : h1;
-        if (hh >= p.H) continue;
-        const uint4 gv = ld_l1_v4(gr + hh);
-        const uint4 yv = *reinterpret_cast<const uint4*>(yr + hh);
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-        uint32_t ov[4];
+    for (int q = 0; q < kCbwdUnroll; ++q) d[q] = 0.0f;
+    for (int c0 = 0; c0 < p.chunks; c0 += kCbwdUnroll) {
+      uint4 gv[kCbwdUnroll][2], yv[kCbwdUnroll][2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
-          d = fmaf(g0, bf16_lo(yw[i]), d);
-          d = fmaf(g1, bf16_hi(yw[i]), d);
-          ov[i] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
+      for (int q = 0; q < kCbwdUnroll; ++q) {
+        const int h0 = piece_channel(c0 + q, lane), h1 = h0 + kHalfChunk;
+        gv[q][0] = gv[q][1] = yv[q][0] = yv[q][1] = make_uint4(0, 0, 0, 0);
+        if (c0 + q < p.chunks) {
+          if (!RAGGED || h0 < p.H) {
+            gv[q][0] = ld_l1_v4(gr + h0);
+            yv[q][0] = *reinterpret_cast<const uint4*>(yr + h0);
+          }
+          if (!RAGGED || h1 < p.H) {
+            gv[q][1] = ld_l1_v4(gr + h1);
+            yv[q][1] = *reinterpret_cast<const uint4*>(yr + h1);
+          }
         }
-        st_v4(dr + hh, make_uint4(ov[0], ov[1], ov[2], ov[3]));
+      }
+#pragma unroll
+      for (int q = 0; q < kCbwdUnroll; ++q) {
+        const int h0 = piece_channel(c0 + q, lane), h1 = h0 + kHalfChunk;
+        uint4 ov[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t gw[4] = {gv[q][h].x, gv[q][h].y, gv[q][h].z, gv[q][h].w};
+          const uint32_t yw[4] = {yv[q][h].x, yv[q][h].y, yv[q][h].z, yv[q][h].w};
+          uint32_t o4[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
+            d[q] = fmaf(g0, bf16_lo(yw[i]), d[q]);
+            d[q] = fmaf(g1, bf16_hi(yw[i]), d[q]);
+            o4[i] = pack_bf16x2(__fmul_rn(w, g0), __fmul_rn(w, g1));
+          }
+          ov[h] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+        if (c0 + q < p.chunks) {
+          if (!RAGGED || h0 < p.H) st_v4(dr + h0, ov[0]);
+          if (!RAGGED || h1 < p.H) st_v4(dr + h1, ov[1]);
+        }
       }
     }
+    float dot = (d[0] + d[1]) + (d[2] + d[3]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-    if (lane == 0) grad_w[u] = d;
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (lane == 0) grad_w[u] = dot;
   }
 }
 
