@@ -57,16 +57,18 @@ def call_bytes(w) -> dict:
 
 # DRAM bytes per launch of the dominant kernel, from a full-size ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum; see profiles/).  An entry only
-# holds for the kernel sources it was taken on: if their hash differs, the
-# bench reports traffic as null.
+# holds for the kernel sources and the launch configuration (the host file
+# picks the grids) it was taken on: if their hash differs, the bench reports
+# traffic as null.
 MEASURED_TRAFFIC = {
     ("prefill", 32768, "combine_backward"): {
         "bytes": 4.23e9 + 3.70e9,
-        "sources_sha1": "3ad17ff065069ece68cd7402e219ae70395a65c5",
+        "sources_sha1": "d7e0c24ade3f85a9d981fc6aae73eefd4f287108",
     },
 }
 KERNEL_SOURCES = ("combine_ep_get_histogram_b200/csrc/common.cuh",
-                  "combine_ep_get_histogram_b200/csrc/movement.cuh")
+                  "combine_ep_get_histogram_b200/csrc/movement.cuh",
+                  "combine_ep_get_histogram_b200/csrc/ep_api.cu")
 
 
 def code_lines(text: str) -> str:

@@ -224,6 +224,32 @@ int movement_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t uni
   return static_cast<int>(need < cap ? need : cap);
 }
 
+// Tokens per CTA of the bulk-store dispatch on the whole GPU (ep_dispatch).
+constexpr int64_t kTmaTokensPerCta = 2;
+
+// The budget is the whole GPU (no SM budget in force).
+bool whole_gpu(const DeviceInfo& d, const ep_shape_t* s) { return s->num_sms <= 0 || s->num_sms >= d.sms; }
+
+// Combine backward on the whole GPU at 16 tokens per SM or more: about
+// kCbwdPairsPerWarp pairs per warp, so the block scheduler balances the end of
+// the kernel, never fewer CTAs than the persistent grid.  Measured against the
+// persistent grid at H = 7168: 161 / 163 us at 4096 tokens, 314 / 320 at 8192,
+// 617 / 635 at 16384, 1222 / 1262 at 32768 (and 702 / 723 at H = 4096); at
+// 2048 tokens and below the persistent grid is as fast or faster.  Combine
+// and dispatch backward measured fastest persistent at the prefill shape and
+// keep movement_grid.  Under an SM budget the grid stays persistent: a budget
+// caps the CTAs resident at once, which only a grid of that size guarantees.
+constexpr int64_t kCbwdPairsPerWarp = 2;
+
+int pair_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t tokens, int64_t pairs) {
+  if (!whole_gpu(d, s) || tokens < 16 * static_cast<int64_t>(d.sms)) return movement_grid(d, s, occ, pairs);
+  const int64_t need = ceil_div(pairs, kMoveWarps);
+  const int64_t cap = grid_cap(d, s, occ);
+  const int64_t want = ceil_div(pairs, kMoveWarps * kCbwdPairsPerWarp);
+  const int64_t g = want > cap ? want : cap;
+  return static_cast<int>(g < need ? g : need);
+}
+
 static_assert(EP_MAX_PEERS == kMaxPeers, "peer tables of the C ABI and the kernels agree");
 
 // Every owner's buffer given, non-null and aligned to `align` bytes.
@@ -390,11 +416,24 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
       if (cached == 0) cached = occupancy(fn, threads, smem);
       occ = cached;
     }
-    // Large batches run 2 CTAs per SM (fewer row copies in flight per SM
-    // measured faster at 32768 tokens); small ones use every resident slot.
-    if (T >= 16 * static_cast<int64_t>(d->sms) && occ > 2) occ = 2;
-    const int64_t cap = grid_cap(*d, shape, occ);
-    const int grid = static_cast<int>(T < cap ? T : cap);
+    const bool large = T >= 16 * static_cast<int64_t>(d->sms);
+    int grid;
+    if (large && whole_gpu(*d, shape)) {
+      // kTmaTokensPerCta tokens per CTA, all resident slots in use: the block
+      // scheduler refills each slot as a CTA retires, and a CTA's second
+      // token loads while its first is quantised.  Measured against the
+      // persistent grid: 54 / 56 us at 4096 tokens, 194 / 211 at 16384,
+      // 380 / 420 at 32768.  Below 16 tokens per SM the persistent grid is as
+      // fast or faster (a partial last wave costs more than it balances).
+      grid = static_cast<int>(ceil_div(T, kTmaTokensPerCta));
+    } else {
+      // Persistent grid.  Large batches under an SM budget run 2 CTAs per SM
+      // (fewer row copies in flight per SM measured faster at 32768 tokens);
+      // small ones use every resident slot.
+      if (large && occ > 2) occ = 2;
+      const int64_t cap = grid_cap(*d, shape, occ);
+      grid = static_cast<int>(T < cap ? T : cap);
+    }
     if (fp8)
       dispatch_tma_kernel<true><<<grid, threads, smem, s>>>(p, static_cast<const uint16_t*>(x), recv_x, recv_scale,
                                                              recv_weight);
@@ -450,7 +489,7 @@ int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const voi
   const MoveParams p = move_params(shape, handle, topk_weights);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
-  const int grid = movement_grid(*d, shape, d->occ_cbwd[ragged], T * shape->k);
+  const int grid = pair_grid(*d, shape, d->occ_cbwd[ragged], T, T * shape->k);
   const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
   const uint16_t* yp = static_cast<const uint16_t*>(y);
   if (ragged)
@@ -597,6 +636,8 @@ int ep_combine_backward_peers(const ep_shape_t* shape, int32_t rank, const int64
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
+  // persistent: with R ranks emulated side by side on one GPU, oversubscribed
+  // grids measured slower (1210 against 1190 us a step at the prefill shape)
   const int grid = movement_grid(*d, shape, d->occ_peer_cbwd[ragged], static_cast<int64_t>(p.T) * p.k);
   const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
   if (ragged)

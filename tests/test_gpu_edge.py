@@ -1,7 +1,8 @@
 """Edge cases of the CUDA path against the oracle, compared in full:
 masked (-1) and duplicate pairs, out-of-range ids, the empty input, k = 1 and
 the k / E maxima, one rank and one expert per rank, ragged hidden sizes and
-layout tiles, every pair on one expert, a one-SM grid, FP8 rounding ties,
+layout tiles, every pair on one expert, a one-SM grid, large batches on the
+whole GPU and under an SM budget, FP8 rounding ties,
 zeros and subnormal codes, and run-to-run determinism."""
 
 import numpy as np
@@ -124,6 +125,16 @@ def test_empty_input(cuda_device):
 ])
 def test_shapes(cuda_device, T, H, k, E, R, use_fp8):
     run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=T + k))
+
+
+@pytest.mark.parametrize("num_sms", [0, 100])
+@pytest.mark.parametrize("H,use_fp8", [(2176, True), (2560, False)])
+def test_large_batch_whole_gpu_and_budget(cuda_device, H, use_fp8, num_sms):
+    """4096 tokens, past 16 per SM: on the whole GPU (num_sms = 0) dispatch and
+    combine backward launch oversubscribed grids, under an SM budget persistent
+    ones; H = 2176 adds a ragged last chunk.  Both against the oracle in full."""
+    T, k, E, R = 4096, 8, 64, 8
+    run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=11), num_sms=num_sms)
 
 
 def test_all_pairs_on_few_experts(cuda_device):
