@@ -201,6 +201,40 @@ class ClockSampler:
 
 # ------------------------------------------------------------- GPU arm
 
+class CallMarks:
+    """Events at the call boundaries of one step.  Warm (no flush): one event
+    before the first call and one after each, the calls back to back.  Cold:
+    L2 is flushed before each call, outside that call's own pair of events."""
+
+    def __init__(self, marks, flush=None):
+        self.marks, self.flush, self.n = marks, flush, 0
+        if flush is None:
+            self._rec()
+
+    def _rec(self):
+        if self.marks is not None:
+            self.marks[self.n].record()
+        self.n += 1
+
+    def begin(self):
+        if self.flush is not None:
+            self.flush()
+            self._rec()
+
+    def end(self):
+        self._rec()
+
+
+def marks_per_step(ncalls: int, cold: bool) -> int:
+    return 2 * ncalls if cold else ncalls + 1
+
+
+def call_ms(marks, ci: int, cold: bool) -> float:
+    """Duration of call ci from one step's marks (CallMarks layout)."""
+    a, b = (marks[2 * ci], marks[2 * ci + 1]) if cold else (marks[ci], marks[ci + 1])
+    return a.elapsed_time(b)
+
+
 class Path:
     """Device buffers of one workload and one step through the C ABI."""
 
@@ -231,40 +265,39 @@ class Path:
         self.grad_w = torch.empty((w.T, w.k), dtype=torch.float32, device=dev)
         self.grad_x = torch.empty((w.T, w.H), dtype=torch.int16, device=dev)
 
-    def step(self, marks=None, before_back=None, after_combine=None):
+    def step(self, marks=None, before_back=None, after_combine=None, flush=None):
         """One pass of the path.  before_back runs (on the host, at enqueue
         time) between dispatch and combine, after_combine right after combine:
-        hooks for the end-to-end pipeline's stream waits and events."""
+        hooks for the end-to-end pipeline's stream waits and events.  marks and
+        flush: see CallMarks."""
         ep, i = self.ep, self.inp
-        n = 0
-
-        def rec():
-            nonlocal n
-            if marks is not None:
-                marks[n].record()
-            n += 1
-
-        rec()
+        m = CallMarks(marks, flush)
         if self.route:
+            m.begin()
             ep.ep_route_group_limited(self.shape, i["scores"], self.w.n_groups, self.w.topk_groups, i["topk_idx"],
                                       i["topk_weights"])
-            rec()
+            m.end()
+        m.begin()
         ep.ep_get_dispatch_layout(self.shape, i["topk_idx"], self.handle, self.ws)
-        rec()
+        m.end()
+        m.begin()
         ep.ep_dispatch(self.shape, i["x"], i["topk_weights"], self.handle, self.recv_x, self.recv_scale,
                        self.recv_weight)
-        rec()
+        m.end()
         if before_back is not None:
             before_back()
+        m.begin()
         ep.ep_combine(self.shape, i["y"], i["topk_weights"], self.handle, self.out)
         if after_combine is not None:
             after_combine()
-        rec()
+        m.end()
+        m.begin()
         ep.ep_combine_backward(self.shape, i["g"], i["y"], i["topk_weights"], self.handle, self.grad_y,
                                self.grad_w)
-        rec()
+        m.end()
+        m.begin()
         ep.ep_dispatch_backward(self.shape, self.grad_y, self.handle, self.grad_x)
-        rec()
+        m.end()
 
 
 def launches_per_step(w, peers: bool = False) -> int:
@@ -300,22 +333,16 @@ class PeersPath(Path):
         Tl = w.T // w.R
         self.ranks = [(r, slice(r * Tl, (r + 1) * Tl)) for r in range(w.R)]
 
-    def step(self, marks=None, before_back=None, after_combine=None):
+    def step(self, marks=None, before_back=None, after_combine=None, flush=None):
         """One step; every call runs its R ranks on R streams forked from and
         joined back to the current stream, as the ranks of R GPUs would run
-        side by side."""
+        them side by side."""
         import torch
         ep, i, sh, h = self.ep, self.inp, self.shape, self.handle
         cur = torch.cuda.current_stream()
         if not hasattr(self, "rank_streams"):
             self.rank_streams = [torch.cuda.Stream(self.dev) for _ in self.ranks]
-        n = 0
-
-        def rec():
-            nonlocal n
-            if marks is not None:
-                marks[n].record()
-            n += 1
+        m = CallMarks(marks, flush)
 
         def fanout(call):
             fork = torch.cuda.Event()
@@ -328,24 +355,28 @@ class PeersPath(Path):
                 done.record(st)
                 cur.wait_event(done)
 
-        rec()
+        m.begin()
         ep.ep_get_dispatch_layout(sh, i["topk_idx"], h, self.ws)
-        rec()
+        m.end()
+        m.begin()
         fanout(lambda r, tok: ep.ep_dispatch_peers(sh, r, i["topk_idx"], h, i["x"][tok], i["topk_weights"][tok],
                                                    self.rx, self.rs, self.rw))
-        rec()
+        m.end()
         if before_back is not None:
             before_back()
+        m.begin()
         fanout(lambda r, tok: ep.ep_combine_peers(sh, r, i["topk_idx"], h, self.ys, i["topk_weights"][tok],
                                                   self.out[tok]))
         if after_combine is not None:
             after_combine()
-        rec()
+        m.end()
+        m.begin()
         fanout(lambda r, tok: ep.ep_combine_backward_peers(sh, r, i["topk_idx"], h, i["g"][tok], self.ys,
                                                            i["topk_weights"][tok], self.gy, self.grad_w[tok]))
-        rec()
+        m.end()
+        m.begin()
         fanout(lambda r, tok: ep.ep_dispatch_backward_peers(sh, r, i["topk_idx"], h, self.gy, self.grad_x[tok]))
-        rec()
+        m.end()
 
 
 B200_L2_BYTES = 126 * 2**20
@@ -362,9 +393,26 @@ def l2_policy(step_bytes: int, l2_bytes: int) -> tuple:
                   f"region; each step timed on its own)")
 
 
+MOVEMENT_CALLS = ("dispatch", "combine", "combine_backward", "dispatch_backward")
+
+
+def per_call_policy(nb: dict, l2_bytes: int) -> tuple:
+    """(cold, description) for the per-call times: when some movement call
+    moves less than 4x the L2 size, it could read what the call before it left
+    in L2, so every call is timed on its own after an L2 flush; otherwise the
+    calls are timed back to back inside the step."""
+    small = min(nb[c] for c in MOVEMENT_CALLS if c in nb)
+    if small < 4 * l2_bytes:
+        return True, (f"cold: each call timed on its own after {2 * l2_bytes / 2**20:.0f} MiB written to flush "
+                      f"L2, outside its events (the smallest call moves {small / 1e6:.0f} MB, under 4x the L2)")
+    return False, (f"warm: calls back to back in the step (the smallest call moves {small / 1e6:.0f} MB, "
+                   f"{small / l2_bytes:.0f}x the L2)")
+
+
 def bench_config(w, args, world: int, l2_bytes: int = B200_L2_BYTES) -> dict:
     """The JSON line's config: the workload by name and sizes (both arms)."""
-    step_bytes = sum(call_bytes(w)[c] for c in step_calls(args))
+    nb = {c: v for c, v in call_bytes(w).items() if c in step_calls(args)}
+    step_bytes = sum(nb.values())
     return {"workload": f"{w.name}: T={w.T} ({w.R} virtual ranks x {w.T // w.R} tokens), H={w.H}, "
                         f"E={w.E}, k={w.k}, top-{w.topk_groups} of {w.n_groups} groups, "
                         f"{'FP8' if w.use_fp8 else 'BF16'} dispatch + BF16 combine + both backward passes",
@@ -372,6 +420,7 @@ def bench_config(w, args, world: int, l2_bytes: int = B200_L2_BYTES) -> dict:
             "storage": ("e4m3 codes + f32 scales dispatched, bf16 expert rows, outputs and gradients"
                         if w.use_fp8 else "bf16 rows, outputs and gradients"),
             "step_bytes": step_bytes, "l2": l2_policy(step_bytes, l2_bytes)[1],
+            "per_call_l2": per_call_policy(nb, l2_bytes)[1],
             "receive_layout": (f"padded [E][R][{args.max_tokens_per_rank}]" if args.max_tokens_per_rank
                                else "dense [T*k]"),
             "parallelism": (f"replicas x{world}" if world > 1 else
@@ -403,7 +452,8 @@ def run_ours(args, rank, world, local):
     nmarks = len(calls) + 1
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size or B200_L2_BYTES
     flush, _ = l2_policy(step_bytes, l2_bytes)
-    flush_buf = torch.empty(2 * l2_bytes // 4, dtype=torch.int32, device=dev) if flush else None
+    cold, _ = per_call_policy(nb, l2_bytes)
+    flush_buf = torch.empty(2 * l2_bytes // 4, dtype=torch.int32, device=dev) if (flush or cold) else None
 
     def flush_l2(i: int):
         if flush_buf is not None:
@@ -434,12 +484,38 @@ def run_ours(args, rank, world, local):
         for _ in range(args.warmup):
             run_step()
         # per-call breakdown: one replay at a time, events read after each
-        for i in range(min(args.steps, 20)):
+        for i in range(0 if cold else min(args.steps, 20)):
             flush_l2(i)
             run_step()
             torch.cuda.synchronize()
             for ci, c in enumerate(calls):
-                per_call_ms[c].append(gmarks[ci].elapsed_time(gmarks[ci + 1]))
+                per_call_ms[c].append(call_ms(gmarks, ci, False))
+        barrier()
+    if cold:
+        # per-call breakdown with L2 flushed before every call (its own step
+        # graph, or eager launches); the timed steps below stay as they are
+        cmarks = [torch.cuda.Event(enable_timing=True, external=not args.no_graph)
+                  for _ in range(marks_per_step(len(calls), True))]
+
+        def cold_flush():
+            flush_buf.add_(1)
+
+        if args.no_graph:
+            def run_cold():
+                path.step(cmarks, flush=cold_flush)
+        else:
+            cold_graph = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(cold_graph):
+                path.step(cmarks, flush=cold_flush)
+            run_cold = cold_graph.replay
+        for _ in range(2):
+            run_cold()
+        for i in range(min(args.steps, 20)):
+            run_cold()
+            torch.cuda.synchronize()
+            for ci, c in enumerate(calls):
+                per_call_ms[c].append(call_ms(cmarks, ci, True))
         barrier()
 
     # device-timed region: K steps back to back on the launching stream
@@ -468,10 +544,10 @@ def run_ours(args, rank, world, local):
     barrier()
     sampler.mark(t0, t1)
     clocks = sampler.stop()
-    if args.no_graph:
+    if args.no_graph and not cold:
         for m in marks:
             for ci, c in enumerate(calls):
-                per_call_ms[c].append(m[ci].elapsed_time(m[ci + 1]))
+                per_call_ms[c].append(call_ms(m, ci, False))
     local_ms = (sum(a.elapsed_time(b) for a, b in step_events) if flush else e_start.elapsed_time(e_end))
     total_ms = max_over_ranks(local_ms, world, dev)
     ms_per_step = total_ms / args.steps

@@ -46,6 +46,41 @@ def test_l2_statement_follows_the_step_bytes():
     assert flush and "flushed" in text
 
 
+def test_per_call_times_are_cold_when_a_call_fits_a_few_l2s():
+    from combine_ep_get_histogram_b200 import workloads as wl
+    l2 = 126 * 2**20
+    decode = {c: v for c, v in bench.call_bytes(wl.CONFIGS["decode"]).items() if c in bench.MOVEMENT_CALLS}
+    prefill = bench.call_bytes(wl.CONFIGS["prefill"])
+    cold, text = bench.per_call_policy(decode, l2)
+    assert cold and "cold" in text          # decode calls move 75-250 MB
+    cold, text = bench.per_call_policy(prefill, l2)
+    assert not cold and "warm" in text      # the layout's few MB do not count
+    assert bench.marks_per_step(5, True) == 10 and bench.marks_per_step(5, False) == 6
+
+
+def test_call_marks_bracket_each_call():
+    class Ev:
+        def __init__(self, log, i):
+            self.log, self.i = log, i
+
+        def record(self):
+            self.log.append(("mark", self.i))
+
+    for cold in (False, True):
+        log = []
+        marks = [Ev(log, i) for i in range(bench.marks_per_step(2, cold))]
+        m = bench.CallMarks(marks, (lambda: log.append(("flush",))) if cold else None)
+        for c in range(2):
+            m.begin()
+            log.append(("call", c))
+            m.end()
+        if cold:
+            assert log == [("flush",), ("mark", 0), ("call", 0), ("mark", 1),
+                           ("flush",), ("mark", 2), ("call", 1), ("mark", 3)]
+        else:
+            assert log == [("mark", 0), ("call", 0), ("mark", 1), ("call", 1), ("mark", 2)]
+
+
 def test_load_skew_is_max_over_mean_of_the_layout_counts():
     import torch
     from combine_ep_get_histogram_b200 import workloads as wl
