@@ -648,7 +648,8 @@ def run_ours(args, rank, world, local):
                  "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel",
                  "route": "route_aligned_kernel|route_group_limited_kernel"}
     if args.peers:
-        kernel_of.update({"dispatch": "dispatch_peers_kernel", "combine": "gather_reduce_peers_kernel<weighted>",
+        kernel_of.update({"dispatch": "dispatch_tma_peers_kernel" if 4 <= -(-w.H // 512) <= 16
+                          else "dispatch_peers_kernel", "combine": "gather_reduce_peers_kernel<weighted>",
                           "combine_backward": "combine_backward_peers_kernel",
                           "dispatch_backward": "gather_reduce_peers_kernel<unweighted>"})
     ach = per_call[dominant]["GB_s"]

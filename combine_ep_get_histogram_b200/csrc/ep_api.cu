@@ -45,6 +45,7 @@ struct DeviceInfo {
   int occ_disp_bf16 = 0, occ_disp_fp8 = 0;
   int occ_comb[2] = {}, occ_dbwd[2] = {};  // [ragged]
   int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
+  int occ_tma_peers[2][kTmaMaxChunks + 1] = {};  // the same for dispatch_tma_peers_kernel
   int occ_cbwd[2] = {};  // [ragged]
   int occ_peer_disp[2] = {}, occ_peer_gather[2][2] = {}, occ_peer_cbwd[2] = {};  // [fp8], [weighted][ragged], [ragged]
   int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
@@ -229,6 +230,27 @@ constexpr int64_t kTmaTokensPerCta = 2;
 
 // The budget is the whole GPU (no SM budget in force).
 bool whole_gpu(const DeviceInfo& d, const ep_shape_t* s) { return s->num_sms <= 0 || s->num_sms >= d.sms; }
+
+// Grid of the bulk-store dispatch (single-GPU and peer forms) for T tokens
+// at occ resident CTAs per SM.
+int tma_dispatch_grid(const DeviceInfo& d, const ep_shape_t* s, int64_t T, int occ) {
+  const bool large = T >= 16 * static_cast<int64_t>(d.sms);
+  if (large && whole_gpu(d, s)) {
+    // kTmaTokensPerCta tokens per CTA, all resident slots in use: the block
+    // scheduler refills each slot as a CTA retires, and a CTA's second token
+    // loads while its first is quantised.  Measured against the persistent
+    // grid: 54 / 56 us at 4096 tokens, 194 / 211 at 16384, 380 / 420 at
+    // 32768.  Below 16 tokens per SM the persistent grid is as fast or faster
+    // (a partial last wave costs more than it balances).
+    return static_cast<int>(ceil_div(T, kTmaTokensPerCta));
+  }
+  // Persistent grid.  Large batches under an SM budget run 2 CTAs per SM
+  // (fewer row copies in flight per SM measured faster at 32768 tokens);
+  // small ones use every resident slot.
+  if (large && occ > 2) occ = 2;
+  const int64_t cap = grid_cap(d, s, occ);
+  return static_cast<int>(T < cap ? T : cap);
+}
 
 // Combine backward on the whole GPU at 16 tokens per SM or more: about
 // kCbwdPairsPerWarp pairs per warp, so the block scheduler balances the end of
@@ -416,24 +438,7 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
       if (cached == 0) cached = occupancy(fn, threads, smem);
       occ = cached;
     }
-    const bool large = T >= 16 * static_cast<int64_t>(d->sms);
-    int grid;
-    if (large && whole_gpu(*d, shape)) {
-      // kTmaTokensPerCta tokens per CTA, all resident slots in use: the block
-      // scheduler refills each slot as a CTA retires, and a CTA's second
-      // token loads while its first is quantised.  Measured against the
-      // persistent grid: 54 / 56 us at 4096 tokens, 194 / 211 at 16384,
-      // 380 / 420 at 32768.  Below 16 tokens per SM the persistent grid is as
-      // fast or faster (a partial last wave costs more than it balances).
-      grid = static_cast<int>(ceil_div(T, kTmaTokensPerCta));
-    } else {
-      // Persistent grid.  Large batches under an SM budget run 2 CTAs per SM
-      // (fewer row copies in flight per SM measured faster at 32768 tokens);
-      // small ones use every resident slot.
-      if (large && occ > 2) occ = 2;
-      const int64_t cap = grid_cap(*d, shape, occ);
-      grid = static_cast<int>(T < cap ? T : cap);
-    }
+    const int grid = tma_dispatch_grid(*d, shape, T, occ);
     if (fp8)
       dispatch_tma_kernel<true><<<grid, threads, smem, s>>>(p, static_cast<const uint16_t*>(x), recv_x, recv_scale,
                                                              recv_weight);
@@ -589,12 +594,31 @@ int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk
   const int64_t units = static_cast<int64_t>(p.T) * p.chunks;
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   const PeerRows rx = peer_rows(recv_x), rs = peer_rows(recv_scale), rw = peer_rows(recv_weight);
-  if (shape->use_fp8)
+  const bool fp8 = shape->use_fp8 != 0;
+  if (p.chunks >= kTmaMinChunks && p.chunks <= kTmaMaxChunks) {
+    const int threads = p.chunks * kWarp;
+    const size_t smem = tma_smem_layout(shape->H, fp8).total;
+    const void* fn = fp8 ? reinterpret_cast<const void*>(dispatch_tma_peers_kernel<true>)
+                         : reinterpret_cast<const void*>(dispatch_tma_peers_kernel<false>);
+    int occ;
+    {
+      std::lock_guard<std::mutex> lock(g_dev_mu);
+      int& cached = const_cast<DeviceInfo*>(d)->occ_tma_peers[fp8][p.chunks];
+      if (cached == 0) cached = occupancy(fn, threads, smem);
+      occ = cached;
+    }
+    const int grid = tma_dispatch_grid(*d, shape, p.T, occ);
+    if (fp8)
+      dispatch_tma_peers_kernel<true><<<grid, threads, smem, s>>>(p, xs, rx, rs, rw);
+    else
+      dispatch_tma_peers_kernel<false><<<grid, threads, smem, s>>>(p, xs, rx, rs, rw);
+  } else if (fp8) {
     dispatch_peers_kernel<true><<<movement_grid(*d, shape, d->occ_peer_disp[1], units), kMoveThreads, 0, s>>>(
         p, xs, rx, rs, rw);
-  else
+  } else {
     dispatch_peers_kernel<false><<<movement_grid(*d, shape, d->occ_peer_disp[0], units), kMoveThreads, 0, s>>>(
         p, xs, rx, rs, rw);
+  }
   return finish(handle, s);
 }
 

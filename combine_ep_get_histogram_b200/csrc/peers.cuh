@@ -14,16 +14,19 @@
 // its owner's buffer.  Combine and dispatch backward load the owners' rows
 // and reduce them.  Combine backward loads y from, and stores grad_y into,
 // the owners' buffers.  An owner's buffer may be another GPU's memory
-// (NVLink peer addresses).  The kernels use plain loads and stores: no TMA,
-// no multicast.  On one GPU, the owners' buffers are R local allocations, and
-// their concatenation equals the single-GPU receive buffer row for row.
+// (NVLink peer addresses).  The kernels use plain loads and stores, and
+// dispatch TMA bulk stores; nothing loads with TMA or multicasts.  On one
+// GPU, the owners' buffers are R local allocations, and their concatenation
+// equals the single-GPU receive buffer row for row.
 //
-// The kernels follow the single-GPU ones: a warp per (token, 512-channel
-// chunk) for dispatch and the gathers (their k row loads in flight in
-// batches of 8), a warp per pair for combine backward (four chunks at a time,
-// one partial sum each), bounds checked per piece only when H is not a
-// multiple of 512.  Dispatch stores 16-byte pieces rather than TMA rows.
-// Peer links (about 0.8 TB/s per direction) rather than HBM bound them.
+// The kernels follow the single-GPU ones.  Dispatch builds each row once in
+// shared memory and writes it to its owners with TMA bulk copies for 4 to 16
+// chunks (a warp per (token, 512-channel chunk) storing 16-byte pieces for
+// other widths).  The gathers take a warp per (token, chunk), their k row
+// loads in flight in batches of 8; combine backward a warp per pair, four
+// chunks at a time with one partial sum each.  Bounds are checked per piece
+// only when H is not a multiple of 512.  Peer links (about 0.8 TB/s per
+// direction) rather than HBM bound them.
 #pragma once
 
 #include "movement.cuh"
@@ -121,6 +124,110 @@ dispatch_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx,
     if (c == 0 && lane < p.k && my_slot >= 0 && rweight.base[my_owner] != nullptr)
       static_cast<float*>(rweight.base[my_owner])[my_row] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
   }
+}
+
+// Dispatch in the single-GPU kernel's form (dispatch_tma_kernel): a CTA per
+// token and a warp per 512-channel chunk; the E4M3 (or BF16) row is built
+// once in shared memory and leaves as one TMA bulk copy per pair
+// (cp.async.bulk.global.shared::cta, a plain store: no multicast) into its
+// owner's buffer, local or a peer's.  Scales and weights leave by plain
+// stores.  The host launches it for 4 to 16 chunks (1536 < H <= 8192), as on
+// one GPU; the shared-memory stage holds each pair's owner next to its row.
+template <bool FP8>
+__global__ void __launch_bounds__(kTmaMaxChunks * kWarp, 3)
+dispatch_tma_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx, PeerRows rscale,
+                          PeerRows rweight) {
+  extern __shared__ __align__(128) uint8_t tma_smem[];
+  __shared__ int32_t row0[kMaxPeers];
+  __shared__ int32_t owner_stage[2 * kMaxK];
+  load_owner_rows(p, row0);
+  const TmaSmemLayout L = tma_smem_layout(p.H, FP8);
+  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
+  const int h0 = piece_channel(warp, lane), h1 = h0 + kHalfChunk;  // one chunk per warp
+  const bool a0 = h0 < p.H, a1 = h1 < p.H;
+  const int row_bytes = FP8 ? p.H : 2 * p.H;
+
+  uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+  int t = blockIdx.x;
+  if (t < p.T) {
+    const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
+    if (a0) v0 = ld_ro_v4(xr + h0);
+    if (a1) v1 = ld_ro_v4(xr + h1);
+  }
+  for (int it = 0; t < p.T; ++it, t += gridDim.x) {
+    const int stage = it & 1;
+    uint8_t* row = tma_smem + (it % L.stages) * L.row_bytes;
+    int32_t* srow = reinterpret_cast<int32_t*>(tma_smem + L.off_slot) + stage * kMaxK;  // owner's local row
+    int32_t* sowner = owner_stage + stage * kMaxK;
+    float* sw = reinterpret_cast<float*>(tma_smem + L.off_w) + stage * kMaxK;
+    float* sscale = reinterpret_cast<float*>(tma_smem + L.off_scale) + stage * p.G;
+
+    // prefetch the next token of this CTA
+    const int tn = t + gridDim.x;
+    uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+    if (tn < p.T) {
+      const uint16_t* xr = x + static_cast<int64_t>(tn) * p.H;
+      if (a0) n0 = ld_ro_v4(xr + h0);
+      if (a1) n1 = ld_ro_v4(xr + h1);
+    }
+    // the row stage is free once the copies issued L.stages tokens ago have read it
+    if (threadIdx.x == 0) bulk_wait_read_all_but(L.stages - 1);
+    if (warp == 0 && lane < p.k) {
+      int o, r;
+      peer_pair(p, row0, t, lane, o, r);
+      srow[lane] = r;
+      sowner[lane] = o;
+      sw[lane] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
+    }
+    __syncthreads();
+
+    if constexpr (FP8) {
+      float sc0, sc1;
+      const uint2 q0 = quantize_piece(v0, sc0);
+      const uint2 q1 = quantize_piece(v1, sc1);
+      const bool scale_lane = (lane & (kLanesPerGroup - 1)) == 0;
+      if (a0) {
+        *reinterpret_cast<uint2*>(row + h0) = q0;
+        if (scale_lane) sscale[h0 / kGroup] = sc0;
+      }
+      if (a1) {
+        *reinterpret_cast<uint2*>(row + h1) = q1;
+        if (scale_lane) sscale[h1 / kGroup] = sc1;
+      }
+    } else {
+      if (a0) *reinterpret_cast<uint4*>(row + 2 * h0) = v0;
+      if (a1) *reinterpret_cast<uint4*>(row + 2 * h1) = v1;
+    }
+    // make the generic-proxy shared-memory writes visible to the bulk copies
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+
+    if (threadIdx.x == 0) {
+      const uint32_t src = static_cast<uint32_t>(__cvta_generic_to_shared(row));
+      for (int j = 0; j < p.k; ++j) {
+        const int r = srow[j];
+        if (r >= 0)
+          bulk_store_row(static_cast<uint8_t*>(rx.base[sowner[j]]) + static_cast<int64_t>(r) * row_bytes, src,
+                         row_bytes);
+      }
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+    if constexpr (FP8) {
+      for (int i = threadIdx.x; i < p.k * p.G; i += blockDim.x) {
+        const int j = i / p.G, g = i - j * p.G;
+        const int r = srow[j];
+        if (r >= 0) static_cast<float*>(rscale.base[sowner[j]])[static_cast<int64_t>(r) * p.G + g] = sscale[g];
+      }
+    }
+    if (threadIdx.x < p.k) {
+      const int r = srow[threadIdx.x];
+      float* wb = static_cast<float*>(rweight.base[sowner[threadIdx.x]]);
+      if (r >= 0 && wb != nullptr) wb[r] = sw[threadIdx.x];
+    }
+    v0 = n0;
+    v1 = n1;
+  }
+  if (threadIdx.x == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // out[t] = bf16( chain over j of (WEIGHTED ? fmaf(w[t,j], y[slot], acc) : acc + y[slot]) ), acc = +0.0f,

@@ -223,9 +223,10 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
  * the single-GPU receive buffer.  The calls below move this rank's tokens
  * only, and read or write each receive row in its owner's buffer, which may
  * be another GPU's memory (a peer address reachable from this device: CUDA
- * IPC, or memory allocated for symmetric access).  Loads and stores are
- * plain ones, with no TMA and no multicast.  The arithmetic is that of the
- * single-GPU calls, element for element.
+ * IPC, or memory allocated for symmetric access).  Loads are plain ones;
+ * stores are plain ones or, in dispatch for 1536 < H <= 8192, TMA bulk
+ * copies from shared memory.  No TMA load and no multicast.  The arithmetic
+ * is that of the single-GPU calls, element for element.
  *
  * shape: the global problem (T = all ranks' tokens); R <= EP_MAX_PEERS.
  * rank: this process's rank.  topk_idx: [T,k] int64, every rank's ids (the

@@ -32,6 +32,14 @@ CASES = {
     "decode-shape-fp8-8ranks": (wl.CONFIGS["decode"].with_(T=8 * 32), 0.0),
     "masked-pairs-ragged-H": (wl.Workload("ragged", T=96, H=640, k=4, E=32, R=4, use_fp8=False,
                                           routing="group", n_groups=4, topk_groups=2), 0.2),
+    # 4 to 16 chunks: dispatch by TMA bulk copies into the owners' buffers
+    "bulk-bf16-masked": (wl.Workload("bulk", T=256, H=2560, k=8, E=64, R=8, use_fp8=False,
+                                     routing="group", n_groups=8, topk_groups=4), 0.1),
+    "bulk-fp8-ragged-H": (wl.Workload("bulk", T=512, H=2176, k=6, E=48, R=4, use_fp8=True,
+                                      routing="group", n_groups=4, topk_groups=2), 0.15),
+    # 2560 tokens per rank, past 16 per SM: the bulk-copy dispatch on an oversubscribed grid
+    "bulk-fp8-large-batch": (wl.Workload("bulk", T=4 * 2560, H=2176, k=4, E=32, R=4, use_fp8=True,
+                                         routing="group", n_groups=4, topk_groups=2), 0.0),
 }
 
 
