@@ -66,11 +66,38 @@ __device__ __forceinline__ int peer_pair(const PeerParams& p, const int32_t* row
   const int64_t e = p.topk_idx[ug];
   owner = 0;
   row = -1;
-  if (s >= 0) {
-    owner = static_cast<int>(e / p.Er);
+  if (s >= 0) {  // a slot means a valid expert id, below E <= 1024: a 32-bit division
+    owner = static_cast<int>(e) / p.Er;
     row = s - row0[owner];
   }
   return s;
+}
+
+// Per expert, the address global slot 0 would have in its owner's buffer of
+// rows of row_bytes (the owner's base minus its first row times row_bytes, in
+// 64-bit integer arithmetic; only rows inside the buffer are ever formed from
+// it).  Staged in shared memory once per CTA, it puts a pair's row one add
+// from its slot: no division and no second lookup between the id and slot
+// loads and the row loads of the gathers, which resolve the k pairs of a
+// token once per chunk (the division and the owner's first row cost 12 % of
+// the peer combine when each pair took them).  The caller synchronises.
+__device__ __forceinline__ void load_expert_bases(const PeerParams& p, const PeerRows& rows, int row_bytes,
+                                                  unsigned long long* base_of) {
+  const int E = p.Er * p.R;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int o = e / p.Er;
+    base_of[e] = reinterpret_cast<unsigned long long>(rows.base[o]) -
+                 static_cast<unsigned long long>(p.expert_offset[o * p.Er]) * static_cast<unsigned>(row_bytes);
+  }
+}
+
+// Address of the owner's row of this rank's pair (t, j); 0 for a masked pair.
+__device__ __forceinline__ unsigned long long peer_row_addr(const PeerParams& p, const unsigned long long* base_of,
+                                                            int t, int j, int row_bytes) {
+  const int64_t ug = (static_cast<int64_t>(p.t_begin) + t) * p.k + j;
+  const int s = p.slot_of_pair[ug];
+  const int e = static_cast<int>(p.topk_idx[ug]);
+  return s < 0 ? 0ull : base_of[e] + static_cast<unsigned long long>(s) * static_cast<unsigned>(row_bytes);
 }
 
 template <bool FP8>
@@ -235,8 +262,9 @@ dispatch_tma_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows
 template <bool WEIGHTED, bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out) {
-  __shared__ int32_t row0[kMaxPeers];
-  load_owner_rows(p, row0);
+  __shared__ unsigned long long base_of[kMaxE];
+  load_expert_bases(p, y, 2 * p.H, base_of);
+  __syncthreads();
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
@@ -245,10 +273,10 @@ gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out)
     const int c = static_cast<int>(u - static_cast<int64_t>(t) * p.chunks);
     const int h0 = piece_channel(c, lane), h1 = h0 + kHalfChunk;
     const bool a0 = !RAGGED || h0 < p.H, a1 = !RAGGED || h1 < p.H;
-    int my_slot = -1, my_owner = 0, my_row = -1;
+    unsigned long long my_row = 0;  // this lane's pair: the row's address, 0 if masked
     float my_w = 0.0f;
     if (lane < p.k) {
-      my_slot = peer_pair(p, row0, t, lane, my_owner, my_row);
+      my_row = peer_row_addr(p, base_of, t, lane, 2 * p.H);
       if (WEIGHTED) my_w = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
     }
     float acc[16];
@@ -256,26 +284,27 @@ gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out)
     for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
     for (int jb = 0; jb < p.k; jb += 8) {  // all loads of a batch of 8 rows in flight, then the arithmetic
       uint4 v[8][2];
-      int s[8];
+      unsigned long long src[8];
       float w[8];
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
         const int j = (jb + jj) & (kWarp - 1);
-        s[jj] = __shfl_sync(0xffffffffu, my_slot, j);
-        const int o = __shfl_sync(0xffffffffu, my_owner, j);
-        const int row = __shfl_sync(0xffffffffu, my_row, j);
+        src[jj] = __shfl_sync(0xffffffffu, my_row, j);
         w[jj] = __shfl_sync(0xffffffffu, my_w, j);
-        if (jb + jj >= p.k) s[jj] = -1;
+        if (jb + jj >= p.k) src[jj] = 0;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
         v[jj][0] = v[jj][1] = make_uint4(0, 0, 0, 0);
-        if (s[jj] >= 0) {
-          const uint16_t* src = static_cast<const uint16_t*>(y.base[o]) + static_cast<int64_t>(row) * p.H;
-          if (a0) v[jj][0] = *reinterpret_cast<const uint4*>(src + h0);
-          if (a1) v[jj][1] = *reinterpret_cast<const uint4*>(src + h1);
+        if (src[jj] != 0) {
+          const uint16_t* r = reinterpret_cast<const uint16_t*>(src[jj]);
+          if (a0) v[jj][0] = *reinterpret_cast<const uint4*>(r + h0);
+          if (a1) v[jj][1] = *reinterpret_cast<const uint4*>(r + h1);
         }
       }
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
-        if (s[jj] < 0) continue;
+        if (src[jj] == 0) continue;
         float f[16];
         unpack8(v[jj][0], f);
         unpack8(v[jj][1], f + 8);
@@ -299,23 +328,27 @@ template <bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 combine_backward_peers_kernel(PeerParams p, const uint16_t* __restrict__ g, PeerRows y, PeerRows grad_y,
                               float* __restrict__ grad_w) {
-  __shared__ int32_t row0[kMaxPeers];
-  load_owner_rows(p, row0);
+  __shared__ unsigned long long y_of[kMaxE], gy_of[kMaxE];
+  load_expert_bases(p, y, 2 * p.H, y_of);
+  load_expert_bases(p, grad_y, 2 * p.H, gy_of);
+  __syncthreads();
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t npairs = static_cast<int64_t>(p.T) * p.k;
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < npairs;
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int t = static_cast<int>(u / p.k), j = static_cast<int>(u - static_cast<int64_t>(t) * p.k);
-    int o, row;
-    const int s = peer_pair(p, row0, t, j, o, row);
+    const int64_t ug = (static_cast<int64_t>(p.t_begin) + t) * p.k + j;
+    const int s = p.slot_of_pair[ug];
     if (s < 0) {
       if (lane == 0) grad_w[u] = 0.0f;
       continue;
     }
+    const int e = static_cast<int>(p.topk_idx[ug]);
+    const unsigned long long off = static_cast<unsigned long long>(s) * static_cast<unsigned>(2 * p.H);
     const float w = p.topk_weights[u];
     const uint16_t* gr = g + static_cast<int64_t>(t) * p.H;
-    const uint16_t* yr = static_cast<const uint16_t*>(y.base[o]) + static_cast<int64_t>(row) * p.H;
-    uint16_t* dr = static_cast<uint16_t*>(grad_y.base[o]) + static_cast<int64_t>(row) * p.H;
+    const uint16_t* yr = reinterpret_cast<const uint16_t*>(y_of[e] + off);
+    uint16_t* dr = reinterpret_cast<uint16_t*>(gy_of[e] + off);
     float d[kCbwdUnroll];
 #pragma unroll
     for (int q = 0; q < kCbwdUnroll; ++q) d[q] = 0.0f;
