@@ -37,6 +37,11 @@ CASES = {
                                      routing="group", n_groups=8, topk_groups=4), 0.1),
     "bulk-fp8-ragged-H": (wl.Workload("bulk", T=512, H=2176, k=6, E=48, R=4, use_fp8=True,
                                       routing="group", n_groups=4, topk_groups=2), 0.15),
+    # k, E and the owner count at their maxima (k = 32, E = 1024, R = 64): the shared-memory tables full
+    "maxima-bulk-fp8": (wl.Workload("maxima", T=64 * 8, H=2048, k=32, E=1024, R=64, use_fp8=True,
+                                    routing="group", n_groups=8, topk_groups=4), 0.05),
+    "maxima-warp-bf16": (wl.Workload("maxima", T=64 * 4, H=256, k=32, E=1024, R=64, use_fp8=False,
+                                     routing="group", n_groups=8, topk_groups=4), 0.0),
     # 2560 tokens per rank, past 16 per SM: the bulk-copy dispatch on an oversubscribed grid
     "bulk-fp8-large-batch": (wl.Workload("bulk", T=4 * 2560, H=2176, k=4, E=32, R=4, use_fp8=True,
                                          routing="group", n_groups=4, topk_groups=2), 0.0),
