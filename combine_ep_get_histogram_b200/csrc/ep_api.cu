@@ -228,13 +228,18 @@ int movement_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t uni
 // Tokens per CTA of the bulk-store dispatch on the whole GPU (ep_dispatch).
 constexpr int64_t kTmaTokensPerCta = 2;
 
+// From this many tokens per SM on, dispatch and combine backward launch
+// oversubscribed grids on the whole GPU (below it, persistent ones measured
+// as fast or faster).
+constexpr int64_t kOversubscribeTokensPerSm = 16;
+
 // The budget is the whole GPU (no SM budget in force).
 bool whole_gpu(const DeviceInfo& d, const ep_shape_t* s) { return s->num_sms <= 0 || s->num_sms >= d.sms; }
 
 // Grid of the bulk-store dispatch (single-GPU and peer forms) for T tokens
 // at occ resident CTAs per SM.
 int tma_dispatch_grid(const DeviceInfo& d, const ep_shape_t* s, int64_t T, int occ) {
-  const bool large = T >= 16 * static_cast<int64_t>(d.sms);
+  const bool large = T >= kOversubscribeTokensPerSm * d.sms;
   if (large && whole_gpu(d, s)) {
     // kTmaTokensPerCta tokens per CTA, all resident slots in use: the block
     // scheduler refills each slot as a CTA retires, and a CTA's second token
@@ -264,7 +269,7 @@ int tma_dispatch_grid(const DeviceInfo& d, const ep_shape_t* s, int64_t T, int o
 constexpr int64_t kCbwdPairsPerWarp = 2;
 
 int pair_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t tokens, int64_t pairs) {
-  if (!whole_gpu(d, s) || tokens < 16 * static_cast<int64_t>(d.sms)) return movement_grid(d, s, occ, pairs);
+  if (!whole_gpu(d, s) || tokens < kOversubscribeTokensPerSm * d.sms) return movement_grid(d, s, occ, pairs);
   const int64_t need = ceil_div(pairs, kMoveWarps);
   const int64_t cap = grid_cap(d, s, occ);
   const int64_t want = ceil_div(pairs, kMoveWarps * kCbwdPairsPerWarp);

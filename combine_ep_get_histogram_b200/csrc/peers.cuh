@@ -96,8 +96,9 @@ __device__ __forceinline__ unsigned long long peer_row_addr(const PeerParams& p,
                                                             int t, int j, int row_bytes) {
   const int64_t ug = (static_cast<int64_t>(p.t_begin) + t) * p.k + j;
   const int s = p.slot_of_pair[ug];
+  if (s < 0) return 0ull;  // masked (or an id the layout rejected): no table entry is read
   const int e = static_cast<int>(p.topk_idx[ug]);
-  return s < 0 ? 0ull : base_of[e] + static_cast<unsigned long long>(s) * static_cast<unsigned>(row_bytes);
+  return base_of[e] + static_cast<unsigned long long>(s) * static_cast<unsigned>(row_bytes);
 }
 
 template <bool FP8>
