@@ -447,7 +447,6 @@ def run_ours(args, rank, world, local):
     if args.peers and (M or args.route):
         raise SystemExit("--peers runs the dense layout without routing")
     path = PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route)
-    stream = torch.cuda.current_stream()
     nb = {c: v for c, v in call_bytes(w).items() if c in calls}
     step_bytes = sum(nb.values())
     nmarks = len(calls) + 1

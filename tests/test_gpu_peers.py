@@ -5,8 +5,9 @@ outputs, their gradients) are separate allocations.  Each rank calls the
 *_peers entry points for its own tokens only, with peer tables that point at
 all owners' buffers, exactly as it would with other GPUs' memory.  The
 concatenation of the owners' buffers must equal the single-GPU receive
-buffer bit for bit, every rank's outputs must equal the single-GPU outputs
-for its tokens, and grad_w must match the oracle within its tolerance."""
+buffer bit for bit, every rank's outputs (grad_w included) must equal the
+single-GPU outputs for its tokens, and grad_w must match the oracle within
+its tolerance."""
 
 import numpy as np
 import pytest
@@ -113,8 +114,11 @@ def test_ranks_reproduce_the_single_gpu_path(cuda_device, name):
     assert np.array_equal(np.concatenate([bf16_host(o) for o in outs]), out1[:w.T])
     assert np.array_equal(cat(gys).view(np.uint16), bf16_host(gy1)[:n_valid])
     assert np.array_equal(np.concatenate([bf16_host(g) for g in gxs]), gx1[:w.T])
+    got_gw = np.concatenate([g.cpu().numpy() for g in gws])
+    # the same partial sums in the same order as the single-GPU kernel: bit-identical
+    assert np.array_equal(got_gw.view(np.uint32), gw1.cpu().numpy()[:w.T].reshape(got_gw.shape).view(np.uint32))
     _, rgw = oracle.combine_backward(d["g"], y, wts, oracle.layout(idx, w.E, w.R)["slot_of_pair"])
-    ok, worst = grad_w_close(np.concatenate([g.cpu().numpy() for g in gws]), rgw)
+    ok, worst = grad_w_close(got_gw, rgw)
     assert ok, worst
 
 
