@@ -44,3 +44,25 @@ def test_bench_line_has_the_contract_keys(cuda_device):
     load = d["load"]  # load skew from the layout's counts: max over mean, at least 1
     for key in ("tokens_per_expert_max_over_mean", "rows_per_rank_max_over_mean", "tokens_per_rank_max_over_mean"):
         assert load[key] >= 1.0
+
+
+def test_bench_line_for_the_emulated_ranks(cuda_device):
+    """--peers: the R ranks' peer calls, every call timed cold (tiny moves far
+    less than the L2), the peer kernels named, no traffic figure (the stored
+    capture is of the single-GPU kernel)."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "tiny", "--peers", "--steps", "4",
+                        "--warmup", "3", "--no-e2e", "--no-cpu-baseline"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["config"]["parallelism"].startswith("1 GPU, 4 ranks emulated")
+    assert d["config"]["per_call_l2"].startswith("cold")
+    if d["roofline"]["call"] != "layout":  # the layout has no peer form
+        assert "peers_kernel" in d["roofline"]["kernel"]
+    assert d["roofline"]["traffic"] is None
+    # tiny: the one-cluster layout, then 4 calls x 4 ranks, per timed step
+    assert d["gpu_launches"] == (1 + 4 * 4) * 4
+    for call in ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward"):
+        assert d["per_call"][call]["us"] > 0
