@@ -653,7 +653,7 @@ def run_ours(args, rank, world, local):
     kernel_of = {"dispatch": "dispatch_tma_kernel<FP8>" if w.use_fp8 else "dispatch_tma_kernel<BF16>",
                  "combine": "gather_reduce_kernel<weighted>", "combine_backward": "combine_backward_kernel",
                  "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel",
-                 "route": "route_aligned_kernel|route_group_limited_kernel"}
+                 "route": "route_compact_kernel|route_aligned_kernel|route_group_limited_kernel"}
     if args.peers:
         kernel_of.update({"dispatch": "dispatch_tma_peers_kernel" if 4 <= -(-w.H // 512) <= 16
                           else "dispatch_peers_kernel", "combine": "gather_reduce_peers_kernel<weighted>",

@@ -50,6 +50,7 @@ struct DeviceInfo {
   int occ_peer_disp[2] = {}, occ_peer_gather[2][2] = {}, occ_peer_cbwd[2] = {};  // [fp8], [weighted][ragged], [ragged]
   int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
   int occ_route_aligned[6] = {};  // route_aligned_kernel<1, 2, 4, 8, 16, 32>
+  int occ_route_compact[6][5] = {};  // route_compact_kernel<2^i, 2^j>, filled on first use
 };
 
 constexpr int kMaxDevices = 64;
@@ -275,6 +276,28 @@ int pair_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t tokens,
   const int64_t want = ceil_div(pairs, kMoveWarps * kCbwdPairsPerWarp);
   const int64_t g = want > cap ? want : cap;
   return static_cast<int>(g < need ? g : need);
+}
+
+// route_compact_kernel<2^nq_log, 2^nc_log> (nc_log < nq_log <= 5).
+const void* route_compact_fn(int nq_log, int nc_log) {
+  switch (nq_log * 8 + nc_log) {
+    case 8 + 0: return reinterpret_cast<const void*>(route_compact_kernel<2, 1>);
+    case 16 + 0: return reinterpret_cast<const void*>(route_compact_kernel<4, 1>);
+    case 16 + 1: return reinterpret_cast<const void*>(route_compact_kernel<4, 2>);
+    case 24 + 0: return reinterpret_cast<const void*>(route_compact_kernel<8, 1>);
+    case 24 + 1: return reinterpret_cast<const void*>(route_compact_kernel<8, 2>);
+    case 24 + 2: return reinterpret_cast<const void*>(route_compact_kernel<8, 4>);
+    case 32 + 0: return reinterpret_cast<const void*>(route_compact_kernel<16, 1>);
+    case 32 + 1: return reinterpret_cast<const void*>(route_compact_kernel<16, 2>);
+    case 32 + 2: return reinterpret_cast<const void*>(route_compact_kernel<16, 4>);
+    case 32 + 3: return reinterpret_cast<const void*>(route_compact_kernel<16, 8>);
+    case 40 + 0: return reinterpret_cast<const void*>(route_compact_kernel<32, 1>);
+    case 40 + 1: return reinterpret_cast<const void*>(route_compact_kernel<32, 2>);
+    case 40 + 2: return reinterpret_cast<const void*>(route_compact_kernel<32, 4>);
+    case 40 + 3: return reinterpret_cast<const void*>(route_compact_kernel<32, 8>);
+    case 40 + 4: return reinterpret_cast<const void*>(route_compact_kernel<32, 16>);
+    default: return nullptr;
+  }
 }
 
 static_assert(EP_MAX_PEERS == kMaxPeers, "peer tables of the C ABI and the kernels agree");
@@ -556,8 +579,28 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
   const int lanes_per_group = per_group / per_lane;
   const bool on_lanes = shape->E % per_lane == 0 && per_group % per_lane == 0 &&
                         (lanes_per_group & (lanes_per_group - 1)) == 0;
-  const int64_t cap = grid_cap(*d, shape, on_lanes ? d->occ_route_aligned[variant] : d->occ_route[variant]);
   const int64_t need = ceil_div(T, warps);
+  if (on_lanes) {
+    // the chosen groups' experts onto all lanes, when that leaves fewer per lane
+    const int64_t cand = static_cast<int64_t>(topk_groups) * per_group;
+    int nc_log = 0;
+    while ((int64_t{kWarp} << nc_log) < cand) ++nc_log;
+    if (nc_log < variant) {
+      const void* fn = route_compact_fn(variant, nc_log);
+      int occ;
+      {
+        std::lock_guard<std::mutex> lock(g_dev_mu);
+        int& cached = const_cast<DeviceInfo*>(d)->occ_route_compact[variant][nc_log];
+        if (cached == 0) cached = occupancy(fn, kRouteThreads, 0);
+        occ = cached;
+      }
+      const int64_t cap = grid_cap(*d, shape, occ);
+      const int grid = static_cast<int>(need < cap ? need : cap);
+      void* args[] = {&p};
+      return cuda_status(cudaLaunchKernel(fn, dim3(grid), dim3(kRouteThreads), args, 0, s));
+    }
+  }
+  const int64_t cap = grid_cap(*d, shape, on_lanes ? d->occ_route_aligned[variant] : d->occ_route[variant]);
   const int grid = static_cast<int>(need < cap ? need : cap);
   if (on_lanes) {
     switch (variant) {

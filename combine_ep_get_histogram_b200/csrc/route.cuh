@@ -17,14 +17,18 @@
 // the lowest expert index.  The selections compare input scores only, so
 // they are exact; the softmax uses fp32 expf.  Scores must be finite.
 //
-// Two kernels.  route_aligned_kernel serves shapes whose groups fall on lane
-// boundaries (E and the group size multiples of NQ, and a power-of-two
+// Three kernels.  route_aligned_kernel serves shapes whose groups fall on
+// lane boundaries (E and the group size multiples of NQ, and a power-of-two
 // number of lanes per group; 256 experts in 8 groups is one): a group's
 // maximum is the lanes' maxima combined by xor shuffles inside the group's
 // lane segment, a group's rank is counted from one shuffle per group, each
 // lane sorts its candidates once (a bitonic network over 64-bit (key,
 // expert) composites), and a pick takes the largest first key over the
 // warp, the winning lane dropping its first entry.
+// route_compact_kernel is the same with the chosen groups' experts first
+// moved onto all 32 lanes, NC < NQ to a lane, in expert order: each lane
+// then sorts NC composites instead of NQ (top-4 of 8 groups of 32: 4 instead
+// of 8), which measured 18 % faster at 32768 tokens x 256 experts.
 // route_group_limited_kernel serves every other shape: one warp
 // max-reduction per group over per-expert group ids.
 #pragma once
@@ -257,6 +261,107 @@ __global__ void __launch_bounds__(kRouteThreads) route_aligned_kernel(RouteParam
 #pragma unroll
         for (int q = 0; q + 1 < NQ; ++q) c[q] = c[q + 1];
         c[NQ - 1] = 0;
+      }
+    }
+    // softmax of the chosen scores (the first one is the largest)
+    const float my_score = lane < p.k ? route_score(my_key) : 0.0f;
+    const float top = __shfl_sync(0xffffffffu, my_score, 0);
+    const float ex = lane < p.k ? expf(my_score - top) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < p.k) {
+      p.topk_idx[t * p.k + lane] = my_expert;
+      p.topk_weights[t * p.k + lane] = __fdiv_rn(ex, sum);
+    }
+  }
+}
+
+// Groups on lane boundaries as in route_aligned_kernel, and the chosen
+// groups' topk_groups * (E / n_groups) experts moved onto the lanes, NC to a
+// lane (NC a power of two below NQ, at least the candidates over 32), in
+// expert order: lane L takes candidates [L*NC, (L+1)*NC) of the chosen groups
+// listed in ascending group order, which lie in one group and one source
+// lane (NC divides NQ and the group size).  The lowest lane among equal keys
+// still holds the lowest expert, so picks and ties are those of
+// route_aligned_kernel.
+template <int NQ, int NC>
+__global__ void __launch_bounds__(kRouteThreads) route_compact_kernel(RouteParams p) {
+  static_assert(NC < NQ && NQ % NC == 0, "compaction takes fewer candidates per lane");
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int per = p.E / p.n_groups;
+  const int lpg = per / NQ;
+  const int e0 = lane * NQ;
+  const bool has = e0 < p.E;
+  const int my_g = lane / lpg;
+  const int f0 = lane * NC;  // this lane's first place in the list of candidates
+  const bool holds = f0 < p.topk_groups * per;
+  const int cg = f0 / per, x = f0 - cg * per;  // chosen group (by rank in group order) and place in it
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp; t < p.T;
+       t += static_cast<int64_t>(gridDim.x) * (kRouteThreads / kWarp)) {
+    const float* s = p.scores + t * p.E;
+    float v[NQ];
+    if (NQ % 4 == 0 && has && (reinterpret_cast<uintptr_t>(s + e0) & 15) == 0) {
+#pragma unroll
+      for (int q = 0; q < NQ; q += 4) {
+        const float4 f = *reinterpret_cast<const float4*>(s + e0 + q);
+        v[q] = f.x;
+        v[q + 1] = f.y;
+        v[q + 2] = f.z;
+        v[q + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) v[q] = has ? s[e0 + q] : 0.0f;
+    }
+    int32_t gk = kRouteNoKey;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) gk = max(gk, has ? route_key(v[q]) : kRouteNoKey);
+    // group maximum over the group's lane segment, and the group's rank
+    for (int o = 1; o < lpg; o <<= 1) gk = max(gk, __shfl_xor_sync(0xffffffffu, gk, o));
+    int rank = 0;
+    for (int g = 0; g < p.n_groups; ++g) {
+      const int32_t other = __shfl_sync(0xffffffffu, gk, g * lpg);
+      rank += (other > gk || (other == gk && g < my_g)) ? 1 : 0;
+    }
+    // the chosen groups' first lanes, and this lane's group among them
+    const unsigned lead = __ballot_sync(0xffffffffu, has && (lane & (lpg - 1)) == 0 && rank < p.topk_groups);
+    unsigned m = lead;
+    for (int i = 0; i < cg; ++i) m &= m - 1;  // drop the cg lower chosen groups
+    const int g = holds ? (__ffs(m) - 1) / lpg : 0;
+    const int ef = g * per + x;  // this lane's first candidate expert
+    const int src = ef / NQ, pos = ef - src * NQ;
+    // fetch scores [pos, pos + NC) of lane src: in round r every lane offers
+    // its scores [r*NC, (r+1)*NC)
+    float nv[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) nv[j] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < NQ / NC; ++r)
+#pragma unroll
+      for (int j = 0; j < NC; ++j) {
+        const float val = __shfl_sync(0xffffffffu, v[r * NC + j], src);
+        if (pos == r * NC) nv[j] = val;
+      }
+    uint64_t c[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) c[j] = holds ? route_composite(route_key(nv[j]), ef + j) : 0;
+    route_sort_desc<NC>(c);
+    int32_t my_key = 0;
+    int my_expert = -1;
+    for (int j = 0; j < p.k; ++j) {
+      const uint32_t head = static_cast<uint32_t>(c[0] >> 32);
+      const uint32_t top = __reduce_max_sync(0xffffffffu, head);
+      const int win = __ffs(__ballot_sync(0xffffffffu, head == top)) - 1;
+      const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(c[0]), win);
+      if (lane == j) {
+        my_key = static_cast<int32_t>(top ^ 0x80000000u);
+        my_expert = static_cast<int>(0xFFFFFFFFu - lo);  // the composite carries the expert itself
+      }
+      if (lane == win) {
+#pragma unroll
+        for (int q = 0; q + 1 < NC; ++q) c[q] = c[q + 1];
+        c[NC - 1] = 0;
       }
     }
     // softmax of the chosen scores (the first one is the largest)

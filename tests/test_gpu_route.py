@@ -1,5 +1,7 @@
-"""Group-limited top-k routing on the GPU against the oracle, through both
-kernels: groups on lane boundaries (the aligned kernel) and off them (the
+"""Group-limited top-k routing on the GPU against the oracle, through the
+three kernels: groups on lane boundaries with the chosen groups' experts
+moved onto all lanes (the compact kernel, whenever that leaves fewer per
+lane) or not (the aligned kernel), and groups off lane boundaries (the
 general kernel).
 
 The selections compare input scores only, so topk_idx must match exactly
@@ -36,14 +38,18 @@ def route_gpu(device, s, k, ng, tg, R=1):
 
 
 @pytest.mark.parametrize("T,E,k,ng,tg", [
-    # groups on lane boundaries
-    (1024, 256, 8, 8, 4),      # decode shape: top-4 of 8 groups, top-8 experts
-    (32768, 256, 8, 8, 4),     # prefill shape
-    (300, 48, 6, 3, 2),        # E not a multiple of 32, 16 experts per group
-    (200, 64, 5, 1, 1),        # one group: plain top-k
-    (77, 256, 3, 32, 1),       # one group of 8 chosen out of 32
-    (512, 1024, 32, 32, 16),   # E and k at their maxima, 32 groups
-    (100, 16, 16, 4, 4),       # every expert chosen
+    # groups on lane boundaries; (experts per lane, candidates per lane) of
+    # the compact kernel in brackets, "aligned" where it would not help
+    (1024, 256, 8, 8, 4),      # decode shape: top-4 of 8 groups, top-8 experts (8, 4)
+    (32768, 256, 8, 8, 4),     # prefill shape (8, 4)
+    (300, 48, 6, 3, 2),        # E not a multiple of 32, 16 experts per group (2, 1)
+    (200, 64, 5, 1, 1),        # one group: plain top-k (aligned)
+    (77, 256, 3, 32, 1),       # one group of 8 chosen out of 32 (8, 1)
+    (512, 1024, 32, 32, 16),   # E and k at their maxima, 32 groups (32, 16)
+    (100, 16, 16, 4, 4),       # every expert chosen (aligned)
+    (333, 512, 8, 16, 4),      # 16 experts per lane (16, 4)
+    (250, 128, 8, 8, 4),       # the backward shape's 128 experts (4, 2)
+    (129, 128, 8, 8, 3),       # 48 candidates: lanes 24 to 31 hold none (4, 2)
     # groups off lane boundaries: 12 experts per group over lanes of 4, 40
     # over lanes of 8, E not a multiple of the experts per lane
     (257, 96, 8, 8, 4),
