@@ -688,6 +688,13 @@ def run_ours(args, rank, world, local):
         "e2e": e2e,
     }
     line["load"] = load
+    if "layout" in per_call and "dispatch" in per_call:
+        # dispatch with and without its layout (the layout is latency-bound and
+        # reported on its own above)
+        us = per_call["layout"]["us"] + per_call["dispatch"]["us"]
+        b = nb["layout"] + nb["dispatch"]
+        line["dispatch_incl_layout"] = {"us": round(us, 2), "bytes": b, "GB_s": round(b / (us * 1e-6) / 1e9, 1),
+                                        "frac_of_peak": round(b / (us * 1e-6) / 1e9 / peak, 3)}
     if overlap is not None:
         line["overlap"] = overlap
     return line

@@ -41,6 +41,8 @@ def test_bench_line_has_the_contract_keys(cuda_device):
     assert d["gpu_launches"] == 5 * 4
     for call in ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward"):
         assert d["per_call"][call]["us"] > 0
+    both = d["dispatch_incl_layout"]  # dispatch with its layout
+    assert abs(both["us"] - d["per_call"]["layout"]["us"] - d["per_call"]["dispatch"]["us"]) < 0.02
     load = d["load"]  # load skew from the layout's counts: max over mean, at least 1
     for key in ("tokens_per_expert_max_over_mean", "rows_per_rank_max_over_mean", "tokens_per_rank_max_over_mean"):
         assert load[key] >= 1.0
