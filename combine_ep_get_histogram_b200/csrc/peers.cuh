@@ -79,8 +79,9 @@ __device__ __forceinline__ int peer_pair(const PeerParams& p, const int32_t* row
 // it).  Staged in shared memory once per CTA, it puts a pair's row one add
 // from its slot: no division and no second lookup between the id and slot
 // loads and the row loads of the gathers, which resolve the k pairs of a
-// token once per chunk (the division and the owner's first row cost 12 % of
-// the peer combine when each pair took them).  The caller synchronises.
+// token once per chunk (the peer combine over all prefill tokens as one
+// launch: 741-751 us with the division and the owner's first row per pair,
+// 661-664 us with the table).  The caller synchronises.
 __device__ __forceinline__ void load_expert_bases(const PeerParams& p, const PeerRows& rows, int row_bytes,
                                                   unsigned long long* base_of) {
   const int E = p.Er * p.R;
