@@ -220,6 +220,14 @@ int finish(const ep_handle_t* h, cudaStream_t stream) {
   return ep_get_error(h, reinterpret_cast<ep_stream_t>(stream));
 }
 
+// finish() for calls without a handle (the router): launch errors, and with
+// EP_DEBUG=1 a synchronisation that surfaces the kernel's own faults.
+int finish_no_handle(cudaStream_t stream) {
+  int st = cuda_status(cudaGetLastError());
+  if (st != EP_OK || !debug_mode()) return st;
+  return cuda_status(cudaStreamSynchronize(stream));
+}
+
 int movement_grid(const DeviceInfo& d, const ep_shape_t* s, int occ, int64_t units_per_warp_grid) {
   const int64_t need = ceil_div(units_per_warp_grid, kMoveWarps);
   const int64_t cap = grid_cap(d, s, occ);
@@ -345,6 +353,18 @@ int peer_setup(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, c
 
 }  // namespace
 
+// Argument checks of ep_get_dispatch_layout other than the workspace, shared
+// with ep_get_dispatch_layout_noalloc (ep_noalloc.cu).  Not exported.
+__attribute__((visibility("hidden"))) int ep_internal_check_layout_args(const ep_shape_t* shape,
+                                                                        const int64_t* topk_idx,
+                                                                        const ep_handle_t* handle) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  if (shape->T > 0 && (topk_idx == nullptr || !aligned(topk_idx, 8))) return EP_ERR_INVALID_ARG;
+  return EP_OK;
+}
+
 extern "C" {
 
 int ep_handle_sizes(const ep_shape_t* shape, int64_t counts[9]) {
@@ -363,11 +383,9 @@ size_t ep_workspace_size(const ep_shape_t* shape) {
 
 int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, const ep_handle_t* handle,
                            void* workspace, size_t workspace_bytes, ep_stream_t stream) {
-  int st = check_shape(shape);
+  int st = ep_internal_check_layout_args(shape, topk_idx, handle);
   if (st != EP_OK) return st;
-  if ((st = check_handle(shape, handle)) != EP_OK) return st;
   const LayoutGeometry g = layout_geometry(shape);
-  if (shape->T > 0 && (topk_idx == nullptr || !aligned(topk_idx, 8))) return EP_ERR_INVALID_ARG;
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < g.total_bytes)
     return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
@@ -400,6 +418,15 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (shape->max_tokens_per_rank > 0) {
     const size_t smem = layout_padded_smem(p.Tr, shape->E, shape->R);
+    if (smem > 48 * 1024) {
+      // a function attribute belongs to the current context (a reset or a
+      // green context starts without it), so it is set before each launch
+      const void* fn = shape->R <= kPadClusterMax ? reinterpret_cast<const void*>(layout_padded_kernel<true>)
+                                                  : reinterpret_cast<const void*>(layout_padded_kernel<false>);
+      if ((st = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem)))) != EP_OK)
+        return st;
+    }
     if (shape->R <= kPadClusterMax) {  // one cluster of R CTAs sums the totals itself
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(shape->R);
@@ -597,7 +624,8 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
       const int64_t cap = grid_cap(*d, shape, occ);
       const int grid = static_cast<int>(need < cap ? need : cap);
       void* args[] = {&p};
-      return cuda_status(cudaLaunchKernel(fn, dim3(grid), dim3(kRouteThreads), args, 0, s));
+      const int launched = cuda_status(cudaLaunchKernel(fn, dim3(grid), dim3(kRouteThreads), args, 0, s));
+      return launched != EP_OK ? launched : finish_no_handle(s);
     }
   }
   const int64_t cap = grid_cap(*d, shape, on_lanes ? d->occ_route_aligned[variant] : d->occ_route[variant]);
@@ -611,7 +639,7 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
       case 4: route_aligned_kernel<16><<<grid, kRouteThreads, 0, s>>>(p); break;
       default: route_aligned_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
     }
-    return cuda_status(cudaGetLastError());
+    return finish_no_handle(s);
   }
   switch (variant) {
     case 0: route_group_limited_kernel<1><<<grid, kRouteThreads, 0, s>>>(p); break;
@@ -621,7 +649,7 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
     case 4: route_group_limited_kernel<16><<<grid, kRouteThreads, 0, s>>>(p); break;
     default: route_group_limited_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
   }
-  return cuda_status(cudaGetLastError());
+  return finish_no_handle(s);
 }
 
 int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, const ep_handle_t* handle,

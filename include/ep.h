@@ -98,7 +98,8 @@ typedef struct {
                       value >= the device's SM count = all SMs; else each of
                       their grids is capped at num_sms x (CTAs of that kernel
                       resident per SM), so the caller's own kernels keep the
-                      rest (blog.hotdry.top, section 二, SM 资源控制).  The
+                      rest ("deepep-expert-parallel-communication-library",
+                      blog.hotdry.top, section 二 SM 资源控制).  The
                       hardware places a grid's CTAs on distinct SMs before it
                       stacks them, so the CTAs land on num_sms SMs only when
                       the stream belongs to an SM partition of that size (a
@@ -171,21 +172,24 @@ int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv,
                          const ep_handle_t* handle, void* grad_x, ep_stream_t stream);
 
 /* ep_get_dispatch_layout without caller-provided scratch.  The pages describe
- * no such call (it has no counterpart there); it exists for callers that
- * cannot allocate device memory: code running while a CUDA graph is being
- * captured, code inside another framework's allocator or memory-pool hooks,
- * and hosts whose device memory is fixed at start-up.  The scratch comes from
- * one fixed array of ep_noalloc_scratch_bytes() (1 MiB) inside the library,
- * which every GPU that loads the library keeps until the process exits.
- *  - Same arguments, results and errors as ep_get_dispatch_layout, minus the
- *    workspace.  Returns EP_ERR_SCRATCH_TOO_SMALL, and enqueues nothing, when
+ * no such call (it has no counterpart there); it exists for callers that may
+ * not allocate device memory: code that runs inside another framework's
+ * allocator or memory-pool hooks (allocating there would re-enter that
+ * allocator), and embedded or real-time hosts whose device memory is fixed
+ * at start-up.  The scratch comes from one fixed array of
+ * ep_noalloc_scratch_bytes() (1 MiB) inside the library, which every GPU that
+ * loads the library keeps until the process exits.
+ *  - Same arguments, results and argument errors as ep_get_dispatch_layout,
+ *    minus the workspace.  After the shape, handle and topk_idx checks, it
+ *    returns EP_ERR_SCRATCH_TOO_SMALL, and enqueues nothing, when
  *    ep_workspace_size(shape) exceeds the array (the limit is about 1000
  *    layout tiles x (E + R) columns, e.g. T = 32768, E = 256, R = 8 needs
  *    271 KiB).
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - The first call in each CUDA context (per device; again after
+ *    cudaDeviceReset, and in each green or driver-API context) looks up the
+ *    array's device address there (cudaGetSymbolAddress) and caches it for
+ *    that context; make that first call before any stream capture.
  *  - Every call on a device shares the one array and leaves its contents
  *    behind; nothing in it needs to start at zero.  Calls whose kernels
  *    overlap on the GPU (other streams, other threads) race on it: order

@@ -88,3 +88,45 @@ def test_route_then_layout(cuda_device):
 def test_route_empty(cuda_device):
     idx, w = route_gpu(cuda_device, np.zeros((0, 64), np.float32), 4, 4, 2)
     assert idx.shape == (0, 4)
+
+
+_DEBUG_SCRIPT = r'''
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+sys.path.insert(0, sys.argv[1] + "/tests")
+import combine_ep_get_histogram_b200 as ep
+import oracle
+from test_gpu_route import scores_for
+dev = torch.device("cuda:0")
+for (T, E, k, ng, tg) in ((1024, 256, 8, 8, 4), (200, 64, 5, 1, 1), (257, 96, 8, 8, 4)):  # the three kernels
+    s = scores_for(T, E, seed=3)
+    sd = torch.from_numpy(s).to(dev)
+    idx = torch.empty((T, k), dtype=torch.int64, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(100_000_000)  # keeps the stream busy for tens of milliseconds
+    ep.ep_route_group_limited(ep.make_shape(T, 128, k, E, 1), sd, ng, tg, idx, w)
+    # with EP_DEBUG=1 the call synchronised the stream before it returned
+    assert torch.cuda.current_stream().query(), "EP_DEBUG=1 did not synchronise the router call"
+    ridx, rw = oracle.route_group_limited(s, k, ng, tg)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=0)
+print("debug ok")
+'''
+
+
+def test_route_under_ep_debug(cuda_device):
+    """EP_DEBUG=1 checks every call, the router's three kernels included: the
+    call returns only after its stream has drained (and reports any error the
+    kernel raised), and the results still match the oracle."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, EP_DEBUG="1")
+    r = subprocess.run([sys.executable, "-c", _DEBUG_SCRIPT, root], capture_output=True, text=True, timeout=300,
+                       env=env)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "debug ok" in r.stdout
