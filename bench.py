@@ -476,23 +476,29 @@ def run_ours(args, rank, world, local):
 
     # One step is captured as a CUDA graph (the C ABI never allocates or
     # synchronises), so small workloads are not timed against Python's call
-    # overhead; events recorded inside the graph mark the call boundaries.
+    # overhead.  The timed graph holds the step's kernels alone; a second
+    # graph of the same step, with events recorded between the calls, gives
+    # the per-call breakdown (event nodes between two kernels add their own
+    # latency and keep a kernel from starting while the previous one drains).
     per_call_ms = {c: [] for c in calls}
     if args.no_graph:
         run_step = path.step
     else:
         gmarks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(nmarks)]
-        graph = torch.cuda.CUDAGraph()
+        graph, mark_graph = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         torch.cuda.synchronize()
         with torch.cuda.graph(graph):
+            path.step()
+        with torch.cuda.graph(mark_graph):
             path.step(gmarks)
         run_step = graph.replay
         for _ in range(args.warmup):
             run_step()
+            mark_graph.replay()
         # per-call breakdown: one replay at a time, events read after each
         for i in range(0 if cold else min(args.steps, 20)):
             flush_l2(i)
-            run_step()
+            mark_graph.replay()
             torch.cuda.synchronize()
             for ci, c in enumerate(calls):
                 per_call_ms[c].append(call_ms(gmarks, ci, False))
@@ -684,7 +690,8 @@ def run_ours(args, rank, world, local):
                      "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, full-size launch"},
         "clocks": clocks,
         "gpu_launches": (launches_per_step(w, args.peers) + (1 if args.route else 0)) * args.steps,
-        "timing": "CUDA graph replay of the step" if not args.no_graph else "eager launches",
+        "timing": ("CUDA graph replay of the step (the kernels alone; the per-call times come from a second graph "
+                   "with events between the calls)" if not args.no_graph else "eager launches"),
         "e2e": e2e,
     }
     line["load"] = load
@@ -837,6 +844,25 @@ def cpu_sample(args, tokens_per_rank: int):
     return ws, d, desc, M
 
 
+def host_cpu() -> dict:
+    """The host the CPU legs run on: the cores this process may use and the
+    CPU model (the oracle itself is single-threaded)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 0
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo", encoding="utf-8", errors="replace") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": cores, "cpu_model": model}
+
+
 def run_cpu_baseline(args) -> dict:
     ws, d, desc, M = cpu_sample(args, args.cpu_tokens_per_rank)
     t = time.perf_counter()
@@ -844,7 +870,7 @@ def run_cpu_baseline(args) -> dict:
     dt = time.perf_counter() - t
     gbs = sum(call_bytes(ws)[c] for c in step_calls(args)) / dt / 1e9
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
-            "seconds": round(dt, 2)}
+            "seconds": round(dt, 2), **host_cpu()}
 
 
 def run_reference(args) -> dict:
@@ -862,8 +888,11 @@ def run_reference(args) -> dict:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32",
-        "data": "synthetic (seeded)", "config": bench_config(workload(args), args, 1),
-        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "data": "synthetic (seeded)",
+        # the configuration this arm actually runs: the sample, and what it is cut from
+        "config": {**bench_config(ws, args, 1), "sample_of": bench_config(workload(args), args, 1)["workload"]},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+                         **host_cpu()},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

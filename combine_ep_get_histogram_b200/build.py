@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libep_b200.so")
-SOURCES = ["ep_api.cu", "ep_noalloc.cu"]
+SOURCES = ["ep_api.cu", "ep_noalloc.cu", "ep_ipc.cu"]
 DEPS = ["common.cuh", "layout.cuh", "movement.cuh", "peers.cuh", "route.cuh"]
 
 NVCC_FLAGS = [

@@ -31,7 +31,8 @@ EXPORTED = ("ep_handle_sizes", "ep_workspace_size", "ep_get_dispatch_layout", "e
             "ep_combine", "ep_combine_backward", "ep_dispatch_backward", "ep_get_error",
             "ep_status_string", "ep_last_cuda_error", "ep_get_dispatch_layout_noalloc",
             "ep_noalloc_scratch_bytes", "ep_route_group_limited", "ep_dispatch_peers", "ep_combine_peers",
-            "ep_combine_backward_peers", "ep_dispatch_backward_peers")
+            "ep_combine_backward_peers", "ep_dispatch_backward_peers", "ep_ipc_export", "ep_ipc_open",
+            "ep_ipc_close")
 
 EP_MAX_PEERS = 64
 
@@ -47,6 +48,10 @@ class ep_handle_t(ctypes.Structure):
 
 class ep_peer_rows_t(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_void_p * EP_MAX_PEERS)]
+
+
+class ep_ipc_buffer_t(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64), ("bytes", ctypes.c_uint64)]
 
 
 class EPError(RuntimeError):
@@ -88,6 +93,9 @@ def _lib():
             "ep_combine_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, pp, vp, vp, vp]),
             "ep_combine_backward_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, vp, pp, vp, pp, vp, vp]),
             "ep_dispatch_backward_peers": (ctypes.c_int, [shp, ctypes.c_int32, vp, hp, pp, vp, vp]),
+            "ep_ipc_export": (ctypes.c_int, [vp, ctypes.POINTER(ep_ipc_buffer_t)]),
+            "ep_ipc_open": (ctypes.c_int, [ctypes.POINTER(ep_ipc_buffer_t), ctypes.POINTER(vp), ctypes.POINTER(vp)]),
+            "ep_ipc_close": (ctypes.c_int, [vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -284,3 +292,32 @@ def ep_dispatch_backward_peers(shape: ep_shape_t, rank: int, topk_idx, handle: H
     st = _lib().ep_dispatch_backward_peers(ctypes.byref(shape), rank, _ptr(topk_idx), ctypes.byref(handle.c),
                                            _byref(peer_rows(grad_recv)), _ptr(grad_x), _stream(stream))
     return _check(st, "ep_dispatch_backward_peers") if check else st
+
+
+# ------------------------------------------- peer buffers between processes (CUDA IPC)
+
+def ep_ipc_export(buf) -> bytes:
+    """The record (ep_ipc_buffer_t, 80 bytes) another process opens to reach
+    this device buffer (a tensor or a raw pointer inside a cudaMalloc
+    allocation)."""
+    rec = ep_ipc_buffer_t()
+    _check(_lib().ep_ipc_export(_ptr(buf), ctypes.byref(rec)), "ep_ipc_export")
+    return bytes(rec)
+
+
+def ep_ipc_open(record: bytes) -> tuple[int, int]:
+    """Maps another process's exported buffer: (mapped_base for
+    ep_ipc_close, the buffer's device address)."""
+    rec = ep_ipc_buffer_t.from_buffer_copy(record)
+    base, ptr = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(_lib().ep_ipc_open(ctypes.byref(rec), ctypes.byref(base), ctypes.byref(ptr)), "ep_ipc_open")
+    return int(base.value), int(ptr.value)
+
+
+def ep_ipc_close(mapped_base: int) -> int:
+    return _check(_lib().ep_ipc_close(mapped_base), "ep_ipc_close")
+
+
+def ipc_record_bytes(record: bytes) -> int:
+    """Bytes from the exported buffer's start to the end of its allocation."""
+    return int(ep_ipc_buffer_t.from_buffer_copy(record).bytes)

@@ -41,3 +41,62 @@ def owner_rows(expert_offset, E: int, R: int) -> list[tuple[int, int]]:
     er = E // R
     off = [int(v) for v in expert_offset]
     return [(off[o * er], off[(o + 1) * er] - off[o * er]) for o in range(R)]
+
+
+class PeerBuffers:
+    """Every rank's copy of a set of named device buffers, for the peer
+    tables of the *_peers calls: this rank's own tensors, and the other
+    ranks' buffers opened through CUDA IPC (ep_ipc_export / ep_ipc_open of
+    the C ABI).
+
+    Collective over `group` (a torch.distributed group, gloo is enough): every
+    rank passes buffers under the same names.  One all-gather of the
+    80-byte export records, then each rank maps the others' buffers.
+    ``table(name)`` lists the device addresses in rank order, this rank's own
+    entry being its local pointer.  ``close()`` unmaps every buffer this rank
+    opened and then waits for the other ranks at a barrier, so that once it
+    returns no rank maps anyone's buffers any more and each rank may free its
+    own.  Until then every rank keeps its local tensors alive."""
+
+    def __init__(self, local: dict, group=None):
+        import torch.distributed as dist
+        from . import ep
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        mine = {n: (ep.ep_ipc_export(t), t.numel() * t.element_size()) for n, t in local.items()}
+        everyone = [None] * self.world
+        dist.all_gather_object(everyone, mine, group=group)
+        self._bases = []
+        self.ptrs = {}
+        try:
+            for name, t in local.items():
+                row = []
+                for r in range(self.world):
+                    if r == self.rank:
+                        row.append(t.data_ptr())
+                        continue
+                    record, nbytes = everyone[r][name]
+                    if ep.ipc_record_bytes(record) < nbytes:
+                        raise ValueError(f"rank {r}'s {name}: the exported allocation is smaller than the buffer")
+                    base, ptr = ep.ep_ipc_open(record)
+                    self._bases.append(base)
+                    row.append(ptr)
+                self.ptrs[name] = row
+        except Exception:
+            self._unmap()
+            raise
+
+    def table(self, name: str) -> list:
+        return self.ptrs[name]
+
+    def _unmap(self):
+        from . import ep
+        while self._bases:
+            ep.ep_ipc_close(self._bases.pop())
+
+    def close(self):
+        import torch.distributed as dist
+        self._unmap()
+        self.ptrs = {}
+        dist.barrier(group=self.group)

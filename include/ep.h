@@ -260,6 +260,44 @@ int ep_dispatch_backward_peers(const ep_shape_t* shape, int32_t rank, const int6
                                const ep_handle_t* handle, const ep_peer_rows_t* grad_recv, void* grad_x,
                                ep_stream_t stream);
 
+/* Peer buffers between processes (one process per GPU, or several on one
+ * GPU): how a rank obtains the addresses of the other ranks' buffers for the
+ * peer tables above, through CUDA IPC.  The EP world is built from a process
+ * group ("DeepEP：MoE 专家并行 EP 通信 kernel 编译与使用指南", section 五
+ * 使用方法), and inside one node the ranks reach each other's memory directly
+ * ("deepep-expert-parallel-communication-library", section 四).  Host calls
+ * only: nothing is enqueued and nothing is allocated.
+ *
+ * ep_ipc_export: describes the device buffer at `ptr` (any address inside a
+ * cudaMalloc allocation of the calling process, e.g. a tensor of torch's
+ * default caching allocator; not stream-ordered pool or virtual-memory
+ * allocations, which give EP_ERR_CUDA) as a plain 80-byte record that can be
+ * sent to the other processes (handle of the whole allocation, the buffer's
+ * offset in it, and the bytes from there to the allocation's end).  The
+ * exporting process keeps the allocation alive, and does not free or reuse
+ * it, until every importer has closed its mapping.
+ * ep_ipc_open: maps another process's exported buffer into this process (on
+ * this process's current device; the exporter's GPU may be another one with
+ * peer access, or the same one) and returns the mapping's base, to be given
+ * to ep_ipc_close, and the buffer's address in it, for the peer tables.  A
+ * process must not open its own export.  Opening the same allocation again
+ * returns the same mapping; each open needs its own close.
+ * ep_ipc_close: unmaps one open (its mapped_base), after the last kernel that
+ * reads or writes through it has finished.
+ *
+ * Ordering between ranks (a buffer's writers before its readers) stays the
+ * caller's: for example, every rank synchronises its stream and then meets
+ * the others at a host barrier between dispatch and combine. */
+typedef struct {
+  unsigned char handle[64]; /* cudaIpcMemHandle_t of the allocation */
+  uint64_t offset;          /* the buffer's byte offset inside the allocation */
+  uint64_t bytes;           /* bytes from the buffer's start to the allocation's end */
+} ep_ipc_buffer_t;
+
+int ep_ipc_export(const void* ptr, ep_ipc_buffer_t* out);
+int ep_ipc_open(const ep_ipc_buffer_t* buf, void** mapped_base, void** ptr);
+int ep_ipc_close(void* mapped_base);
+
 /* Synchronises `stream`, reads handle->error_word, clears it, and returns
  * EP_ERR_BAD_INDEX if a bad expert id was seen since the last read, else
  * EP_ERR_CAPACITY if a padded block overflowed, else EP_OK; EP_ERR_CUDA if

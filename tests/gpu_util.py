@@ -116,15 +116,33 @@ def grad_w_close(got: np.ndarray, ref: np.ndarray, rel=1e-2):
     return bool(np.all(ok)), float(np.max(err / np.maximum(np.abs(ref), rms)) if ref.size else 0.0)
 
 
-def sample_tokens(T: int, R: int, n: int, seed: int = 123) -> np.ndarray:
-    """Random tokens plus the first and last token of every virtual rank."""
-    if T == 0:
-        return np.zeros(0, np.int64)
-    rng = np.random.default_rng(seed)
-    Tr = T // R
-    edges = np.concatenate([np.arange(R) * Tr, np.arange(1, R + 1) * Tr - 1])
-    pick = rng.choice(T, size=min(n, T), replace=False)
-    return np.unique(np.concatenate([edges, pick]))
+def oracle_threads() -> int:
+    """Host threads for the chunked oracle comparisons (the oracle's C calls
+    release the GIL, so chunks run in parallel)."""
+    import os
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(32, n))
+
+
+def compare_in_chunks(T: int, chunk: int, fetch, check, threads: int | None = None):
+    """Every token in [0, T) in chunks of `chunk`: fetch(t0, t1) reads the GPU
+    outputs of the chunk on the calling thread, check(t0, t1, fetched) runs the
+    oracle on the chunk and compares, on a thread pool.  At most two chunks per
+    thread are held at once, so host memory stays bounded at any T."""
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or oracle_threads()
+    with ThreadPoolExecutor(threads) as ex:
+        pending = []
+        for t0 in range(0, T, chunk):
+            t1 = min(T, t0 + chunk)
+            pending.append(ex.submit(check, t0, t1, fetch(t0, t1)))
+            if len(pending) >= 2 * threads:
+                pending.pop(0).result()
+        for f in pending:
+            f.result()
 
 
 class StepBuffers:

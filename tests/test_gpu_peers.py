@@ -3,11 +3,14 @@
 Every owner rank's receive buffers (dispatch payload, scales, weights, expert
 outputs, their gradients) are separate allocations.  Each rank calls the
 *_peers entry points for its own tokens only, with peer tables that point at
-all owners' buffers, exactly as it would with other GPUs' memory.  The
-concatenation of the owners' buffers must equal the single-GPU receive
-buffer bit for bit, every rank's outputs (grad_w included) must equal the
-single-GPU outputs for its tokens, and grad_w must match the oracle within
-its tolerance."""
+all owners' buffers, exactly as it would with other GPUs' memory.
+
+Every output is compared with the CPU oracle directly: the concatenation of
+the owners' buffers with the oracle's receive buffer (payload, scales,
+weights, grad_y), every rank's combined tokens and grad_x with the oracle's
+combine and dispatch backward, grad_w within its tolerance.  The outputs are
+also bit-identical to the single-GPU path's (the same arithmetic, element for
+element, in the same order)."""
 
 import numpy as np
 import pytest
@@ -17,7 +20,7 @@ import combine_ep_get_histogram_b200 as ep
 import oracle
 from combine_ep_get_histogram_b200 import multi
 from combine_ep_get_histogram_b200 import workloads as wl
-from gpu_util import GpuPath, bf16_host, grad_w_close, to_dev
+from gpu_util import GpuPath, assert_bits_equal, bf16_host, grad_w_close, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -117,9 +120,24 @@ def test_ranks_reproduce_the_single_gpu_path(cuda_device, name):
     got_gw = np.concatenate([g.cpu().numpy() for g in gws])
     # the same partial sums in the same order as the single-GPU kernel: bit-identical
     assert np.array_equal(got_gw.view(np.uint32), gw1.cpu().numpy()[:w.T].reshape(got_gw.shape).view(np.uint32))
-    _, rgw = oracle.combine_backward(d["g"], y, wts, oracle.layout(idx, w.E, w.R)["slot_of_pair"])
+
+    # every output against the oracle
+    lay = oracle.layout(idx, w.E, w.R)
+    assert np.array_equal(lay["expert_offset"], eoff)
+    slots = lay["slot_of_pair"]
+    orx, ors, orw = oracle.dispatch(d["x"], wts, slots, w.use_fp8)
+    got_rx = cat(rx)
+    assert_bits_equal("peer recv_x", got_rx if w.use_fp8 else got_rx.view(np.uint16), orx[:n_valid])
+    assert_bits_equal("peer recv_weight", cat(rw).view(np.uint32), orw[:n_valid].view(np.uint32))
+    if w.use_fp8:
+        assert_bits_equal("peer recv_scale", cat(rs).view(np.uint32), ors[:n_valid].view(np.uint32))
+    assert_bits_equal("peer combine out", np.concatenate([bf16_host(o) for o in outs]), oracle.combine(y, wts, slots))
+    rgy, rgw = oracle.combine_backward(d["g"], y, wts, slots)
+    assert_bits_equal("peer grad_y", cat(gys).view(np.uint16), rgy[:n_valid])
     ok, worst = grad_w_close(got_gw, rgw)
     assert ok, worst
+    assert_bits_equal("peer grad_x", np.concatenate([bf16_host(g) for g in gxs]),
+                      oracle.dispatch_backward(rgy, slots, w.T, w.k))
 
 
 def test_one_rank_is_the_single_gpu_path(cuda_device):
@@ -133,3 +151,7 @@ def test_one_rank_is_the_single_gpu_path(cuda_device):
     ep.ep_dispatch_peers(one.shape, 0, one.idx, one.handle, to_dev(d["x"], cuda_device), one.wts, [rx], None, [rw])
     torch.cuda.synchronize()
     assert torch.equal(rx, rx1) and torch.equal(rw, rw1)
+    orx, _, orw = oracle.dispatch(d["x"], d["topk_weights"], oracle.layout(d["topk_idx"], w.E, w.R)["slot_of_pair"],
+                                  False)
+    assert_bits_equal("R=1 recv_x", bf16_host(rx), orx)
+    assert_bits_equal("R=1 recv_weight", rw.cpu().numpy().view(np.uint32), orw.view(np.uint32))

@@ -82,12 +82,17 @@ def test_reference_arm_prints_on_rank_zero_only():
         assert key in line, key
     assert line["n_gpus"] == 2 and line["steps"] == 1 and line["warmup"] == 3
     assert line["higher_is_better"] is True and line["unit"] == line["e2e"]["unit"] == "GB/s"
-    # the same workload and config as the GPU arm's line
-    assert line["config"]["workload"].startswith("prefill: T=32768") and line["config"]["H"] == 7168
-    nb = bench.call_bytes(bench.workload(_default_args()))
+    # the config is the sample this arm ran (2 tokens per rank of the prefill
+    # shape), and names the GPU arm's workload it is cut from
+    assert line["config"]["workload"].startswith("prefill: T=16 ") and line["config"]["T"] == 16
+    assert line["config"]["H"] == 7168 and line["config"]["sample_of"].startswith("prefill: T=32768")
+    sample = bench.workload(_default_args()).with_(T=16)
+    nb = bench.call_bytes(sample)
     assert line["config"]["step_bytes"] == sum(nb[c] for c in bench.CALLS)
-    for key in ("value", "unit", "cores", "kind", "sample"):
+    assert "T=16 " in line["cpu_baseline"]["sample"]
+    for key in ("value", "unit", "cores", "kind", "sample", "host_cores", "cpu_model"):
         assert key in line["cpu_baseline"], key
+    assert line["cpu_baseline"]["host_cores"] >= 1 and line["cpu_baseline"]["cores"] == 1
 
 
 def _default_args():

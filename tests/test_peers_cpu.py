@@ -86,3 +86,99 @@ def test_token_range_and_owner_rows_reject_uneven_splits():
         multi.token_range(10, 4, 0)
     with pytest.raises(ValueError):
         multi.owner_rows([0] * 11, 10, 4)
+
+
+class _FakeBuf:
+    """Stands in for a device tensor: an address and a size, nothing else."""
+
+    def __init__(self, ptr, n):
+        self.ptr, self.n = ptr, n
+
+    def data_ptr(self):
+        return self.ptr
+
+    def numel(self):
+        return self.n
+
+    def element_size(self):
+        return 4
+
+
+def _peer_buffers_main(rank, world, port, q, short):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from combine_ep_get_histogram_b200 import ep, multi
+    opened, closed = [], []
+
+    # host-side fakes of the C ABI's IPC calls: a record names the exporter's
+    # address and the bytes its allocation holds from there
+    def export(t):
+        nbytes = t.numel() * t.element_size()
+        if short and rank == 1 and t.ptr % 1000 == 2:
+            nbytes -= 4  # rank 1 claims an allocation too small for its "b" buffer
+        return f"{t.data_ptr()}:{nbytes}".encode()
+
+    def record_bytes(rec):
+        return int(rec.decode().split(":")[1])
+
+    def open_(rec):
+        ptr = int(rec.decode().split(":")[0])
+        opened.append(ptr + 5)
+        return ptr + 5, ptr + 7
+
+    ep.ep_ipc_export, ep.ipc_record_bytes, ep.ep_ipc_open = export, record_bytes, open_
+    ep.ep_ipc_close = closed.append
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        local = {"a": _FakeBuf(10_000 * (rank + 1) + 1, 16), "b": _FakeBuf(10_000 * (rank + 1) + 2, 8)}
+        try:
+            pb = multi.PeerBuffers(local)
+        except ValueError as e:
+            q.put((rank, "refused", str(e), sorted(opened), sorted(closed)))
+            dist.barrier()
+            return
+        tables = {n: pb.table(n) for n in local}
+        pb.close()
+        q.put((rank, "ok", tables, sorted(opened), sorted(closed)))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_peer_buffers(short):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_peer_buffers_main, args=(r, world, port, q, short)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    return sorted(q.get(timeout=10) for _ in range(world))
+
+
+def test_peer_buffers_tables_and_close():
+    """Each rank's table lists every rank's buffer in rank order: its own
+    local address, the others' through the opened mappings; close() unmaps
+    every mapping it opened."""
+    res = _run_peer_buffers(short=False)
+    for rank, status, tables, opened, closed in res:
+        assert status == "ok"
+        for name, off in (("a", 1), ("b", 2)):
+            expect = [10_000 * (r + 1) + off + (0 if r == rank else 7) for r in range(3)]
+            assert tables[name] == expect
+        assert len(opened) == 2 * 2 and opened == closed
+
+
+def test_peer_buffers_refuse_a_short_allocation():
+    """A peer whose exported allocation cannot hold the buffer is refused,
+    and whatever was already mapped is unmapped."""
+    res = _run_peer_buffers(short=True)
+    for rank, status, msg, opened, closed in res:
+        if rank == 1:
+            assert status == "ok" or status == "refused"
+        else:
+            assert status == "refused" and "rank 1" in msg
+            assert opened == closed
