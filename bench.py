@@ -794,6 +794,16 @@ def measure_overlap(args, w, d, dev, M, step_ms):
 def workload(args):
     from combine_ep_get_histogram_b200 import workloads as wl
     w = wl.CONFIGS[args.workload]
+    # reshaped workloads (profiling captures of the other kernel variants)
+    if getattr(args, "ranks", 0):
+        w = w.with_(T=w.T // w.R * args.ranks, R=args.ranks)
+    if getattr(args, "hidden", 0):
+        w = w.with_(H=args.hidden)
+    if getattr(args, "experts", 0):
+        w = w.with_(E=args.experts)
+    if getattr(args, "groups", 0):
+        w = w.with_(routing="group", n_groups=args.groups,
+                    topk_groups=getattr(args, "topk_groups", 0) or min(w.topk_groups, args.groups))
     if args.tokens_per_rank:
         w = w.with_(T=w.R * args.tokens_per_rank)
     if args.dispatch_dtype != "default":
@@ -912,6 +922,11 @@ def main():
                     help="override the workload's dispatch payload (the skewed workload is timed with both)")
     ap.add_argument("--tokens-per-rank", type=int, default=0,
                     help="resize the workload to R x this many tokens (profiling captures)")
+    ap.add_argument("--hidden", type=int, default=0, help="reshape: hidden size H (profiling captures)")
+    ap.add_argument("--experts", type=int, default=0, help="reshape: number of experts E")
+    ap.add_argument("--groups", type=int, default=0, help="reshape: expert groups of the group-limited routing")
+    ap.add_argument("--topk-groups", type=int, default=0, help="reshape: groups each token picks")
+    ap.add_argument("--ranks", type=int, default=0, help="reshape: virtual ranks R (same tokens per rank)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each call eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")

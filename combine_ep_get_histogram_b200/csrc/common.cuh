@@ -107,6 +107,34 @@ __device__ __forceinline__ uint2 pack8_e4m3(const float* f) {
                     pack_e4m3x2(f[4], f[5]) | (pack_e4m3x2(f[6], f[7]) << 16));
 }
 
+// Programmatic dependent launch.  The host launches every kernel of the
+// library with programmatic stream serialization (unless EP_PDL=0), and
+// every kernel opens with the same three steps:
+//   1. pdl_allow_next(): the next kernel on the stream may be scheduled now,
+//      so its CTAs take SM slots as this grid's CTAs retire, instead of after
+//      the last one;
+//   2. optional L2 prefetches of the lines the kernel reads first: a prefetch
+//      writes nothing and returns nothing to the thread, so it is harmless
+//      while the previous kernel may still be writing those lines;
+//   3. pdl_wait_prev(): blocks until the previous kernel on the stream has
+//      completed and its memory writes are visible.
+// Every global load and store of a kernel comes after step 3, so a kernel
+// never reads data its predecessor has not finished writing, and never
+// overwrites data its predecessor may still read.  Without the launch
+// attribute both instructions do nothing.
+__device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Brings the 128-byte lines of [p, p + bytes) into L2, one line per thread
+// (thread `tid` of `nthreads`).  Every address lies inside the range.
+__device__ __forceinline__ void prefetch_l2(const void* p, int64_t bytes, int tid, int nthreads) {
+  if (bytes <= 0) return;
+  const char* c = static_cast<const char*>(p);
+  const int64_t first = reinterpret_cast<uintptr_t>(c) & 127;  // offset of p in its line
+  for (int64_t off = static_cast<int64_t>(tid) * 128 - first; off < bytes; off += static_cast<int64_t>(nthreads) * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(c + (off < 0 ? 0 : off)));
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

@@ -202,8 +202,9 @@ LayoutGeometry layout_geometry(const ep_shape_t* s) {
   return g;
 }
 
-MoveParams move_params(const ep_shape_t* s, const ep_handle_t* h, const float* w) {
+MoveParams move_params(const ep_shape_t* s, const ep_handle_t* h, const float* w, bool pdl) {
   MoveParams p;
+  p.pdl = pdl ? 1 : 0;
   p.T = s->T;
   p.H = s->H;
   p.k = s->k;
@@ -218,6 +219,43 @@ int finish(const ep_handle_t* h, cudaStream_t stream) {
   int st = cuda_status(cudaGetLastError());
   if (st != EP_OK || !debug_mode()) return st;
   return ep_get_error(h, reinterpret_cast<ep_stream_t>(stream));
+}
+
+// Programmatic dependent launch (common.cuh): on unless EP_PDL=0.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* s = std::getenv("EP_PDL");
+    return !(s != nullptr && s[0] == '0');
+  }();
+  return on;
+}
+
+// Fills the programmatic-serialization launch attribute (when `pdl`) at
+// attrs[n] and returns the new attribute count.
+unsigned pdl_attribute(cudaLaunchAttribute* attrs, unsigned n, bool pdl) {
+  if (!pdl) return n;
+  attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[n].val.programmaticStreamSerializationAllowed = 1;
+  return n + 1;
+}
+
+// kernel<<<grid, block, smem, s>>>(args...), with programmatic stream
+// serialization when `pdl`: the kernel may be scheduled while the previous
+// kernel on the stream drains, and waits for it (griddepcontrol.wait) before
+// any global access.  Launch errors are left for finish() to read, as with
+// <<<>>>.
+template <typename... KArgs, typename... Args>
+void launch(bool pdl, void (*kernel)(KArgs...), int64_t grid, int block, size_t smem, cudaStream_t s,
+            Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[1];
+  cfg.numAttrs = pdl_attribute(attrs, 0, pdl);
+  cfg.attrs = attrs;
+  (void)cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 // finish() for calls without a handle (the router): launch errors, and with
@@ -241,6 +279,16 @@ constexpr int64_t kTmaTokensPerCta = 2;
 // oversubscribed grids on the whole GPU (below it, persistent ones measured
 // as fast or faster).
 constexpr int64_t kOversubscribeTokensPerSm = 16;
+
+// Programmatic dependent launch for a call over `tokens` tokens: only below
+// kOversubscribeTokensPerSm tokens per SM, where the grids are persistent and
+// a call lasts tens of microseconds.  Measured on the decode shape (1024
+// tokens): step 115.6 against 117.7 us without it.  On large batches it cost
+// time instead (prefill step 2929 against 2886 us, backward workload 1832
+// against 1815 us, same GPU), so they launch without it.
+bool use_pdl(const DeviceInfo& d, int64_t tokens) {
+  return pdl_enabled() && tokens < kOversubscribeTokensPerSm * d.sms;
+}
 
 // The budget is the whole GPU (no SM budget in force).
 bool whole_gpu(const DeviceInfo& d, const ep_shape_t* s) { return s->num_sms <= 0 || s->num_sms >= d.sms; }
@@ -390,6 +438,7 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
     return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, shape->T);
 
   LayoutParams p;
   p.topk_idx = topk_idx;
@@ -433,13 +482,13 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
       cfg.blockDim = dim3(kPadThreads);
       cfg.dynamicSmemBytes = smem;
       cfg.stream = s;
-      cudaLaunchAttribute attr[1];
+      cudaLaunchAttribute attr[2];
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = shape->R;
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
-      cfg.numAttrs = 1;
+      cfg.numAttrs = pdl_attribute(attr, 1, pdl);
       if ((st = cuda_status(cudaLaunchKernelEx(&cfg, layout_padded_kernel<true>, p, shape->max_tokens_per_rank))) !=
           EP_OK)
         return st;
@@ -448,20 +497,20 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
     if ((st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_expert, 0, shape->E * 4, s))) != EP_OK ||
         (st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_rank, 0, shape->R * 4, s))) != EP_OK)
       return st;
-    layout_padded_kernel<false><<<shape->R, kPadThreads, smem, s>>>(p, shape->max_tokens_per_rank);
+    launch(pdl, layout_padded_kernel<false>, shape->R, kPadThreads, smem, s, p, shape->max_tokens_per_rank);
     return finish(handle, s);
   }
   if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
-    layout_small_kernel<<<kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s>>>(p);
+    launch(pdl, layout_small_kernel, kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s, p);
     return finish(handle, s);
   }
   if (g.nt > 0) {
     const size_t smem = static_cast<size_t>(g.ncol) * 4 + static_cast<size_t>(g.tile_t) * shape->R;
-    layout_count_kernel<<<g.nt, kLayoutThreads, smem, s>>>(p);
+    launch(pdl, layout_count_kernel, g.nt, kLayoutThreads, smem, s, p);
   }
-  layout_scan_kernel<<<g.ncol, kLayoutThreads, 0, s>>>(p);
+  launch(pdl, layout_scan_kernel, g.ncol, kLayoutThreads, 0, s, p);
   const size_t smem_assign = static_cast<size_t>(shape->E + 1 + kLayoutWarps * shape->E) * 4;
-  layout_assign_kernel<<<g.nt > 0 ? g.nt : 1, kLayoutThreads, smem_assign, s>>>(p);
+  launch(pdl, layout_assign_kernel, g.nt > 0 ? g.nt : 1, kLayoutThreads, smem_assign, s, p);
   return finish(handle, s);
 }
 
@@ -476,8 +525,9 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
   if (recv_weight != nullptr && !aligned(recv_weight, 4)) return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, T);
   if (T == 0) return EP_OK;
-  const MoveParams p = move_params(shape, handle, topk_weights);
+  const MoveParams p = move_params(shape, handle, topk_weights, pdl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t units = T * p.chunks;
   if (p.chunks >= kTmaMinChunks && p.chunks <= kTmaMaxChunks) {
@@ -495,17 +545,17 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
     }
     const int grid = tma_dispatch_grid(*d, shape, T, occ);
     if (fp8)
-      dispatch_tma_kernel<true><<<grid, threads, smem, s>>>(p, static_cast<const uint16_t*>(x), recv_x, recv_scale,
-                                                             recv_weight);
+      launch(pdl, dispatch_tma_kernel<true>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x, recv_scale,
+          recv_weight);
     else
-      dispatch_tma_kernel<false><<<grid, threads, smem, s>>>(p, static_cast<const uint16_t*>(x), recv_x, nullptr,
-                                                              recv_weight);
+      launch(pdl, dispatch_tma_kernel<false>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x, nullptr,
+          recv_weight);
   } else if (shape->use_fp8) {
-    dispatch_kernel<true><<<movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s>>>(
-        p, static_cast<const uint16_t*>(x), recv_x, recv_scale, recv_weight);
+    launch(pdl, dispatch_kernel<true>, movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s, p,
+        static_cast<const uint16_t*>(x), recv_x, recv_scale, recv_weight);
   } else {
-    dispatch_kernel<false><<<movement_grid(*d, shape, d->occ_disp_bf16, units), kMoveThreads, 0, s>>>(
-        p, static_cast<const uint16_t*>(x), recv_x, nullptr, recv_weight);
+    launch(pdl, dispatch_kernel<false>, movement_grid(*d, shape, d->occ_disp_bf16, units), kMoveThreads, 0, s, p,
+        static_cast<const uint16_t*>(x), recv_x, nullptr, recv_weight);
   }
   return finish(handle, s);
 }
@@ -519,17 +569,18 @@ int ep_combine(const ep_shape_t* shape, const void* y, const float* topk_weights
   if (!rows_ok(y, P) || !rows_ok(out, T) || !f32_ok(topk_weights, P)) return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, T);
   if (T == 0) return EP_OK;
-  const MoveParams p = move_params(shape, handle, topk_weights);
+  const MoveParams p = move_params(shape, handle, topk_weights, pdl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
   const int grid = movement_grid(*d, shape, d->occ_comb[ragged], T * p.chunks);
   if (ragged)
-    gather_reduce_kernel<true, true><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(y),
-                                                                  static_cast<uint16_t*>(out));
+    launch(pdl, gather_reduce_kernel<true, true>, grid, kMoveThreads, 0, s, p, static_cast<const uint16_t*>(y),
+        static_cast<uint16_t*>(out));
   else
-    gather_reduce_kernel<true, false><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(y),
-                                                                   static_cast<uint16_t*>(out));
+    launch(pdl, gather_reduce_kernel<true, false>, grid, kMoveThreads, 0, s, p, static_cast<const uint16_t*>(y),
+        static_cast<uint16_t*>(out));
   return finish(handle, s);
 }
 
@@ -545,17 +596,18 @@ int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const voi
     return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, T);
   if (T == 0) return EP_OK;
-  const MoveParams p = move_params(shape, handle, topk_weights);
+  const MoveParams p = move_params(shape, handle, topk_weights, pdl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
   const int grid = pair_grid(*d, shape, d->occ_cbwd[ragged], T, T * shape->k);
   const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
   const uint16_t* yp = static_cast<const uint16_t*>(y);
   if (ragged)
-    combine_backward_kernel<true><<<grid, kMoveThreads, 0, s>>>(p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
+    launch(pdl, combine_backward_kernel<true>, grid, kMoveThreads, 0, s, p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
   else
-    combine_backward_kernel<false><<<grid, kMoveThreads, 0, s>>>(p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
+    launch(pdl, combine_backward_kernel<false>, grid, kMoveThreads, 0, s, p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
   return finish(handle, s);
 }
 
@@ -568,17 +620,18 @@ int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv, const e
   if (!rows_ok(grad_recv, P) || !rows_ok(grad_x, T)) return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, T);
   if (T == 0) return EP_OK;
-  const MoveParams p = move_params(shape, handle, nullptr);
+  const MoveParams p = move_params(shape, handle, nullptr, pdl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
   const int grid = movement_grid(*d, shape, d->occ_dbwd[ragged], T * p.chunks);
   if (ragged)
-    gather_reduce_kernel<false, true><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_recv),
-                                                                   static_cast<uint16_t*>(grad_x));
+    launch(pdl, gather_reduce_kernel<false, true>, grid, kMoveThreads, 0, s, p, static_cast<const uint16_t*>(grad_recv),
+        static_cast<uint16_t*>(grad_x));
   else
-    gather_reduce_kernel<false, false><<<grid, kMoveThreads, 0, s>>>(p, static_cast<const uint16_t*>(grad_recv),
-                                                                    static_cast<uint16_t*>(grad_x));
+    launch(pdl, gather_reduce_kernel<false, false>, grid, kMoveThreads, 0, s, p, static_cast<const uint16_t*>(grad_recv),
+        static_cast<uint16_t*>(grad_x));
   return finish(handle, s);
 }
 
@@ -594,6 +647,7 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
     return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, T);
   if (T == 0) return EP_OK;
   RouteParams p{scores, shape->T, shape->E, shape->k, n_groups, topk_groups, topk_idx, topk_weights};
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -624,7 +678,14 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
       const int64_t cap = grid_cap(*d, shape, occ);
       const int grid = static_cast<int>(need < cap ? need : cap);
       void* args[] = {&p};
-      const int launched = cuda_status(cudaLaunchKernel(fn, dim3(grid), dim3(kRouteThreads), args, 0, s));
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(kRouteThreads);
+      cfg.stream = s;
+      cudaLaunchAttribute attrs[1];
+      cfg.numAttrs = pdl_attribute(attrs, 0, pdl);
+      cfg.attrs = attrs;
+      const int launched = cuda_status(cudaLaunchKernelExC(&cfg, fn, args));
       return launched != EP_OK ? launched : finish_no_handle(s);
     }
   }
@@ -632,22 +693,22 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
   const int grid = static_cast<int>(need < cap ? need : cap);
   if (on_lanes) {
     switch (variant) {
-      case 0: route_aligned_kernel<1><<<grid, kRouteThreads, 0, s>>>(p); break;
-      case 1: route_aligned_kernel<2><<<grid, kRouteThreads, 0, s>>>(p); break;
-      case 2: route_aligned_kernel<4><<<grid, kRouteThreads, 0, s>>>(p); break;
-      case 3: route_aligned_kernel<8><<<grid, kRouteThreads, 0, s>>>(p); break;
-      case 4: route_aligned_kernel<16><<<grid, kRouteThreads, 0, s>>>(p); break;
-      default: route_aligned_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
+      case 0: launch(pdl, route_aligned_kernel<1>, grid, kRouteThreads, 0, s, p); break;
+      case 1: launch(pdl, route_aligned_kernel<2>, grid, kRouteThreads, 0, s, p); break;
+      case 2: launch(pdl, route_aligned_kernel<4>, grid, kRouteThreads, 0, s, p); break;
+      case 3: launch(pdl, route_aligned_kernel<8>, grid, kRouteThreads, 0, s, p); break;
+      case 4: launch(pdl, route_aligned_kernel<16>, grid, kRouteThreads, 0, s, p); break;
+      default: launch(pdl, route_aligned_kernel<32>, grid, kRouteThreads, 0, s, p); break;
     }
     return finish_no_handle(s);
   }
   switch (variant) {
-    case 0: route_group_limited_kernel<1><<<grid, kRouteThreads, 0, s>>>(p); break;
-    case 1: route_group_limited_kernel<2><<<grid, kRouteThreads, 0, s>>>(p); break;
-    case 2: route_group_limited_kernel<4><<<grid, kRouteThreads, 0, s>>>(p); break;
-    case 3: route_group_limited_kernel<8><<<grid, kRouteThreads, 0, s>>>(p); break;
-    case 4: route_group_limited_kernel<16><<<grid, kRouteThreads, 0, s>>>(p); break;
-    default: route_group_limited_kernel<32><<<grid, kRouteThreads, 0, s>>>(p); break;
+    case 0: launch(pdl, route_group_limited_kernel<1>, grid, kRouteThreads, 0, s, p); break;
+    case 1: launch(pdl, route_group_limited_kernel<2>, grid, kRouteThreads, 0, s, p); break;
+    case 2: launch(pdl, route_group_limited_kernel<4>, grid, kRouteThreads, 0, s, p); break;
+    case 3: launch(pdl, route_group_limited_kernel<8>, grid, kRouteThreads, 0, s, p); break;
+    case 4: launch(pdl, route_group_limited_kernel<16>, grid, kRouteThreads, 0, s, p); break;
+    default: launch(pdl, route_group_limited_kernel<32>, grid, kRouteThreads, 0, s, p); break;
   }
   return finish_no_handle(s);
 }
@@ -665,6 +726,7 @@ int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk
   if (shape->use_fp8 && p.T > 0 && !peer_rows_ok(recv_scale, R, 4)) return EP_ERR_INVALID_ARG;
   if (recv_weight != nullptr && p.T > 0 && !peer_rows_ok(recv_weight, R, 4)) return EP_ERR_INVALID_ARG;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, p.T);
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t units = static_cast<int64_t>(p.T) * p.chunks;
@@ -685,15 +747,15 @@ int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk
     }
     const int grid = tma_dispatch_grid(*d, shape, p.T, occ);
     if (fp8)
-      dispatch_tma_peers_kernel<true><<<grid, threads, smem, s>>>(p, xs, rx, rs, rw);
+      launch(pdl, dispatch_tma_peers_kernel<true>, grid, threads, smem, s, p, xs, rx, rs, rw);
     else
-      dispatch_tma_peers_kernel<false><<<grid, threads, smem, s>>>(p, xs, rx, rs, rw);
+      launch(pdl, dispatch_tma_peers_kernel<false>, grid, threads, smem, s, p, xs, rx, rs, rw);
   } else if (fp8) {
-    dispatch_peers_kernel<true><<<movement_grid(*d, shape, d->occ_peer_disp[1], units), kMoveThreads, 0, s>>>(
-        p, xs, rx, rs, rw);
+    launch(pdl, dispatch_peers_kernel<true>, movement_grid(*d, shape, d->occ_peer_disp[1], units), kMoveThreads, 0, s, p, xs,
+        rx, rs, rw);
   } else {
-    dispatch_peers_kernel<false><<<movement_grid(*d, shape, d->occ_peer_disp[0], units), kMoveThreads, 0, s>>>(
-        p, xs, rx, rs, rw);
+    launch(pdl, dispatch_peers_kernel<false>, movement_grid(*d, shape, d->occ_peer_disp[0], units), kMoveThreads, 0, s, p,
+        xs, rx, rs, rw);
   }
   return finish(handle, s);
 }
@@ -707,15 +769,17 @@ int ep_combine_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk_
   if (topk_weights == nullptr && p.T > 0) return EP_ERR_INVALID_ARG;
   if (!rows_ok(out, p.T) || (p.T > 0 && !peer_rows_ok(y, shape->R, 16))) return EP_ERR_INVALID_ARG;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, p.T);
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
   const int grid = movement_grid(*d, shape, d->occ_peer_gather[1][ragged], static_cast<int64_t>(p.T) * p.chunks);
   if (ragged)
-    gather_reduce_peers_kernel<true, true><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(y), static_cast<uint16_t*>(out));
+    launch(pdl, gather_reduce_peers_kernel<true, true>, grid, kMoveThreads, 0, s, p, peer_rows(y),
+        static_cast<uint16_t*>(out));
   else
-    gather_reduce_peers_kernel<true, false><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(y),
-                                                                         static_cast<uint16_t*>(out));
+    launch(pdl, gather_reduce_peers_kernel<true, false>, grid, kMoveThreads, 0, s, p, peer_rows(y),
+        static_cast<uint16_t*>(out));
   return finish(handle, s);
 }
 
@@ -733,6 +797,7 @@ int ep_combine_backward_peers(const ep_shape_t* shape, int32_t rank, const int64
       (p.T > 0 && (!peer_rows_ok(y, R, 16) || !peer_rows_ok(grad_y, R, 16))))
     return EP_ERR_INVALID_ARG;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, p.T);
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
@@ -741,10 +806,11 @@ int ep_combine_backward_peers(const ep_shape_t* shape, int32_t rank, const int64
   const int grid = movement_grid(*d, shape, d->occ_peer_cbwd[ragged], static_cast<int64_t>(p.T) * p.k);
   const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
   if (ragged)
-    combine_backward_peers_kernel<true><<<grid, kMoveThreads, 0, s>>>(p, gp, peer_rows(y), peer_rows(grad_y), grad_w);
+    launch(pdl, combine_backward_peers_kernel<true>, grid, kMoveThreads, 0, s, p, gp, peer_rows(y), peer_rows(grad_y),
+        grad_w);
   else
-    combine_backward_peers_kernel<false><<<grid, kMoveThreads, 0, s>>>(p, gp, peer_rows(y), peer_rows(grad_y),
-                                                                      grad_w);
+    launch(pdl, combine_backward_peers_kernel<false>, grid, kMoveThreads, 0, s, p, gp, peer_rows(y), peer_rows(grad_y),
+        grad_w);
   return finish(handle, s);
 }
 
@@ -757,16 +823,17 @@ int ep_dispatch_backward_peers(const ep_shape_t* shape, int32_t rank, const int6
   if (st != EP_OK) return st;
   if (!rows_ok(grad_x, p.T) || (p.T > 0 && !peer_rows_ok(grad_recv, shape->R, 16))) return EP_ERR_INVALID_ARG;
   if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, p.T);
   if (p.T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool ragged = shape->H % kChunk != 0;
   const int grid = movement_grid(*d, shape, d->occ_peer_gather[0][ragged], static_cast<int64_t>(p.T) * p.chunks);
   if (ragged)
-    gather_reduce_peers_kernel<false, true><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(grad_recv),
-                                                                         static_cast<uint16_t*>(grad_x));
+    launch(pdl, gather_reduce_peers_kernel<false, true>, grid, kMoveThreads, 0, s, p, peer_rows(grad_recv),
+        static_cast<uint16_t*>(grad_x));
   else
-    gather_reduce_peers_kernel<false, false><<<grid, kMoveThreads, 0, s>>>(p, peer_rows(grad_recv),
-                                                                          static_cast<uint16_t*>(grad_x));
+    launch(pdl, gather_reduce_peers_kernel<false, false>, grid, kMoveThreads, 0, s, p, peer_rows(grad_recv),
+        static_cast<uint16_t*>(grad_x));
   return finish(handle, s);
 }
 

@@ -79,6 +79,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutPara
   bool bad = false;
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t* idx = p.topk_idx + static_cast<int64_t>(t0) * p.k;
+  pdl_allow_next();
+  prefetch_l2(idx, static_cast<int64_t>(npairs) * 8, threadIdx.x, blockDim.x);
+  pdl_wait_prev();
   // a tile holds at most kTilePairs pairs: every thread loads its (up to)
   // kPairsPerThread expert ids first, then counts them
   int e[kPairsPerThread];
@@ -159,6 +162,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scan_kernel(LayoutParam
   __shared__ int32_t scratch[kWarp];
   const int c = blockIdx.x;
   int32_t* col = p.colhist + static_cast<int64_t>(c) * p.nt;
+  pdl_allow_next();
+  pdl_wait_prev();
   const int32_t total = block_exclusive_scan(col, p.nt, scratch);
   if (threadIdx.x == 0) p.coltotal[c] = total;
   if (c < p.E) {
@@ -196,6 +201,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
   const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
   int ereg[kMaxChunksPerWarp];
   bool bad = false;  // already reported by layout_count_kernel
+  pdl_allow_next();
+  pdl_wait_prev();
 #pragma unroll
   for (int c = 0; c < kMaxChunksPerWarp; ++c) {
     const int i = my_lo + c * kWarp + lane;
@@ -335,6 +342,9 @@ layout_small_kernel(LayoutParams p) {
 
   bool bad = false;
   int ereg[kSmallChunks];
+  pdl_allow_next();
+  prefetch_l2(p.topk_idx + pair0, static_cast<int64_t>(npairs) * 8, threadIdx.x, blockDim.x);
+  pdl_wait_prev();
 #pragma unroll
   for (int q = 0; q < kSmallChunks; ++q) {
     const int i = my_lo + q * kWarp + lane;
@@ -508,6 +518,9 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
 
   bool bad = false, over = false;
   int ereg[kPadChunks];
+  pdl_allow_next();
+  prefetch_l2(p.topk_idx + pair0, static_cast<int64_t>(npairs) * 8, threadIdx.x, blockDim.x);
+  pdl_wait_prev();
 #pragma unroll
   for (int q = 0; q < kPadChunks; ++q) {
     const int i = my_lo + q * kWarp + lane;

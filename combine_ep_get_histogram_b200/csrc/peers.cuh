@@ -8,8 +8,9 @@
 // keeps the rows [expert_offset[o*E/R], expert_offset[(o+1)*E/R]) of the
 // global receive buffer, and slot s is its local row s - expert_offset[o*E/R].
 // The kernels fuse the exchange with the arithmetic (the pages' dispatch and
-// combine are all-to-alls between ranks: zhouruolin.cn, section 五; the
-// normal kernels move tokens over NVLink: blog.hotdry.top, section 一).
+// combine are all-to-alls between ranks: "DeepEP：MoE 专家并行 EP 通信 kernel
+// 编译与使用指南", section 五; the normal kernels move tokens over NVLink:
+// "deepep-expert-parallel-communication-library", section 一).
 // Dispatch quantises this rank's tokens and stores each row straight into
 // its owner's buffer.  Combine and dispatch backward load the owners' rows
 // and reduce them.  Combine backward loads y from, and stores grad_y into,
@@ -106,6 +107,8 @@ template <bool FP8>
 __global__ void __launch_bounds__(kMoveThreads)
 dispatch_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows rx, PeerRows rscale, PeerRows rweight) {
   __shared__ int32_t row0[kMaxPeers];
+  pdl_allow_next();
+  pdl_wait_prev();
   load_owner_rows(p, row0);
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
@@ -169,6 +172,8 @@ dispatch_tma_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows
   extern __shared__ __align__(128) uint8_t tma_smem[];
   __shared__ int32_t row0[kMaxPeers];
   __shared__ int32_t owner_stage[2 * kMaxK];
+  pdl_allow_next();
+  pdl_wait_prev();
   load_owner_rows(p, row0);
   const TmaSmemLayout L = tma_smem_layout(p.H, FP8);
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
@@ -265,6 +270,8 @@ template <bool WEIGHTED, bool RAGGED>
 __global__ void __launch_bounds__(kMoveThreads)
 gather_reduce_peers_kernel(PeerParams p, PeerRows y, uint16_t* __restrict__ out) {
   __shared__ unsigned long long base_of[kMaxE];
+  pdl_allow_next();
+  pdl_wait_prev();
   load_expert_bases(p, y, 2 * p.H, base_of);
   __syncthreads();
   const int lane = threadIdx.x & (kWarp - 1);
@@ -331,6 +338,8 @@ __global__ void __launch_bounds__(kMoveThreads)
 combine_backward_peers_kernel(PeerParams p, const uint16_t* __restrict__ g, PeerRows y, PeerRows grad_y,
                               float* __restrict__ grad_w) {
   __shared__ unsigned long long y_of[kMaxE], gy_of[kMaxE];
+  pdl_allow_next();
+  pdl_wait_prev();
   load_expert_bases(p, y, 2 * p.H, y_of);
   load_expert_bases(p, grad_y, 2 * p.H, gy_of);
   __syncthreads();

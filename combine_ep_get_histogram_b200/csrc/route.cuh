@@ -3,7 +3,8 @@
 //
 // The pages describe group-limited gating in words: experts are split into
 // groups, a token first picks its best groups and then its top-k experts
-// inside them ("top-4 groups, top-8 experts": blog.hotdry.top, sections 一
+// inside them ("top-4 groups, top-8 experts":
+// "deepep-expert-parallel-communication-library", sections 一
 // and 三).  Reading taken where they are silent: a group's score is the
 // largest score of its experts; groups and experts are chosen by descending
 // score with ties to the lower index; topk_idx lists the experts by
@@ -59,11 +60,22 @@ constexpr int32_t kRouteNoKey = INT32_MIN;  // below every finite score's key
 
 // NQ = experts per lane (E <= 32*NQ); the caller picks the smallest of
 // 1, 2, 4, 8, 16, 32 that holds E.
+// Programmatic-launch prologue of the router kernels (common.cuh): let the
+// next kernel be scheduled, bring the warp's first score row into L2, then
+// wait for the previous kernel's writes.
+__device__ __forceinline__ void route_prologue(const RouteParams& p) {
+  pdl_allow_next();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp;
+  if (t0 < p.T) prefetch_l2(p.scores + t0 * p.E, 4 * static_cast<int64_t>(p.E), threadIdx.x & (kWarp - 1), kWarp);
+  pdl_wait_prev();
+}
+
 template <int NQ>
 __global__ void __launch_bounds__(kRouteThreads) route_group_limited_kernel(RouteParams p) {
   const int lane = threadIdx.x & (kWarp - 1);
   const int per = p.E / p.n_groups;
   const int e0 = lane * NQ;
+  route_prologue(p);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp; t < p.T;
        t += static_cast<int64_t>(gridDim.x) * (kRouteThreads / kWarp)) {
     const float* s = p.scores + t * p.E;
@@ -207,6 +219,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_aligned_kernel(RouteParam
   const int e0 = lane * NQ;
   const bool has = e0 < p.E;
   const int my_g = lane / lpg;
+  route_prologue(p);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp; t < p.T;
        t += static_cast<int64_t>(gridDim.x) * (kRouteThreads / kWarp)) {
     const float* s = p.scores + t * p.E;
@@ -297,6 +310,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_compact_kernel(RouteParam
   const int f0 = lane * NC;  // this lane's first place in the list of candidates
   const bool holds = f0 < p.topk_groups * per;
   const int cg = f0 / per, x = f0 - cg * per;  // chosen group (by rank in group order) and place in it
+  route_prologue(p);
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * (kRouteThreads / kWarp) + threadIdx.x / kWarp; t < p.T;
        t += static_cast<int64_t>(gridDim.x) * (kRouteThreads / kWarp)) {
     const float* s = p.scores + t * p.E;

@@ -7,12 +7,13 @@ binding nor the CPU oracle, so both can be fed from it.
 The workload shapes follow the pages' own benchmark setups: 4096 tokens per
 rank, hidden 7168, top-4 groups and top-8 experts, FP8 dispatch and BF16
 combine for the "normal" (training / prefill) kernels, and 128 tokens per rank,
-hidden 7168, top-8 for the low-latency decode kernels (blog.hotdry.top,
-"deepep-expert-parallel-communication-library", section 一 两种内核设计; the
-czhn.yksolo.com article "DeepSeek 开源周第二弹", sections 具有 NVLink 和 RDMA
-转发的普通内核 and 具有纯 RDMA 的低延迟内核).  Group-limited gating (experts
-split into groups; a token first picks groups, then experts inside them) is
-the routing those pages describe (blog.hotdry.top, section 三 NVLink-RDMA
+hidden 7168, top-8 for the low-latency decode kernels
+("deepep-expert-parallel-communication-library" (blog.hotdry.top), section 一
+两种内核设计; "DeepSeek 开源周第二弹" (czhn.yksolo.com), sections 具有 NVLink
+和 RDMA 转发的普通内核 and 具有纯 RDMA 的低延迟内核).  Group-limited gating
+(experts split into groups; a token first picks groups, then experts inside
+them) is the routing those pages describe
+("deepep-expert-parallel-communication-library", section 三 NVLink-RDMA
 跨域转发).  No public dataset is used by the pages; these synthetic draws stand
 in for real router traces.
 

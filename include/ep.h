@@ -8,17 +8,17 @@
  *    returns the received tokens, their gate weights and a handle; combine
  *    brings the experts' outputs back to each token's rank and sums them
  *    using that handle; the same handle serves combine_backward and
- *    dispatch_backward ("DeepEP：MoE 专家并行 EP 通信 kernel 编译与使用指南",
- *    zhouruolin.cn, section 五 使用方法 and FAQ Q5).
+ *    dispatch_backward ("DeepEP：MoE 专家并行 EP 通信 kernel 编译与使用指南"
+ *    (zhouruolin.cn), section 五 使用方法 and FAQ Q5).
  *  - FP8 dispatch with BF16 combine is the standard precision pair
- *    (blog.hotdry.top "deepep-expert-parallel-communication-library",
- *    section 五 实践建议; czhn.yksolo.com "DeepSeek 开源周第二弹": 原生 FP8
+ *    ("deepep-expert-parallel-communication-library" (blog.hotdry.top),
+ *    section 五 实践建议; "DeepSeek 开源周第二弹" (czhn.yksolo.com): 原生 FP8
  *    调度支持), and the precision conversion is fused into the data movement
- *    ("DeepEP：专为MoE模型打造的All-to-All通信库", bjdmk.com.cn, section 3.2).
+ *    ("DeepEP：专为MoE模型打造的All-to-All通信库" (bjdmk.com.cn), section 3.2).
  *  - the per-expert token counts are the quantity one inspects for load skew
- *    (bjdmk.com.cn, section 5.2).
- *  - the number of SMs a call may use is a caller knob (blog.hotdry.top,
- *    section 二 SM 资源控制).
+ *    ("DeepEP：专为MoE模型打造的All-to-All通信库", section 5.2).
+ *  - the number of SMs a call may use is a caller knob
+ *    ("deepep-expert-parallel-communication-library", section 二 SM 资源控制).
  *
  * Model of the expert-parallel world: one GPU, R virtual ranks.  Rank r owns
  * source tokens [r*T/R, (r+1)*T/R) and experts [r*E/R, (r+1)*E/R).  Every
@@ -26,7 +26,8 @@
  * partition is rows [expert_offset[r*E/R], expert_offset[(r+1)*E/R]).  Dense
  * layout: P = T*k rows, no gaps.  Padded layout (the low-latency kernels'
  * static per-expert buffers, sized by num_max_tokens_per_rank, for decoding
- * with CUDA graphs: blog.hotdry.top, sections 一 and 二; zhouruolin.cn,
+ * with CUDA graphs: "deepep-expert-parallel-communication-library",
+ * sections 一 and 二; "DeepEP：MoE 专家并行 EP 通信 kernel 编译与使用指南",
  * section 五): E*R*M rows, see ep_shape_t.max_tokens_per_rank.
  *
  * Numerics (the pages do not fix them; these are the definitions used):
@@ -99,7 +100,7 @@ typedef struct {
                       their grids is capped at num_sms x (CTAs of that kernel
                       resident per SM), so the caller's own kernels keep the
                       rest ("deepep-expert-parallel-communication-library",
-                      blog.hotdry.top, section 二 SM 资源控制).  The
+                      "deepep-expert-parallel-communication-library", section 二 SM 资源控制).  The
                       hardware places a grid's CTAs on distinct SMs before it
                       stacks them, so the CTAs land on num_sms SMs only when
                       the stream belongs to an SM partition of that size (a
@@ -202,8 +203,8 @@ size_t ep_noalloc_scratch_bytes(void);
 
 /* Group-limited top-k routing, the step that produces topk_idx and
  * topk_weights (experts split into groups; a token picks its best groups,
- * then its top-k experts inside them: blog.hotdry.top "deepep-expert-
- * parallel-communication-library", sections 一 and 三).
+ * then its top-k experts inside them: "deepep-expert-parallel-
+ * communication-library", sections 一 and 三).
  * scores: [T,E] fp32, finite, device.  Experts are n_groups groups of E /
  * n_groups consecutive ids (n_groups <= 32); a group's score is its largest
  * expert score; the topk_groups best groups are kept, then the k best
@@ -215,9 +216,10 @@ int ep_route_group_limited(const ep_shape_t* shape, const float* scores, int n_g
 
 /* ---- Multi-GPU expert parallelism: one process per GPU -----------------
  *
- * R ranks, one GPU each (the pages' EP8 over NVLink: blog.hotdry.top
+ * R ranks, one GPU each (the pages' EP8 over NVLink:
  * "deepep-expert-parallel-communication-library", section 一; dispatch and
- * combine are all-to-alls between ranks: zhouruolin.cn, section 五).  Rank r
+ * combine are all-to-alls between ranks: "DeepEP：MoE 专家并行 EP 通信
+ * kernel 编译与使用指南", section 五).  Rank r
  * holds tokens [r*T/R, (r+1)*T/R) and experts [r*E/R, (r+1)*E/R).  Every
  * rank gathers all ranks' topk_idx ([T,k], T*k*8 bytes) and runs
  * ep_get_dispatch_layout over it, so every rank holds the same global

@@ -14,10 +14,11 @@
  *  - per-expert token counts as the load-skew diagnostic: "DeepEP：专为MoE模型
  *    打造的All-to-All通信库" (bjdmk.com.cn), section 5.2.
  *  - FP8 dispatch with BF16 combine as the standard precision pair:
- *    blog.hotdry.top "deepep-expert-parallel-communication-library",
- *    section 五 实践建议; czhn.yksolo.com "DeepSeek 开源周第二弹" (原生 FP8
+ *    "deepep-expert-parallel-communication-library" (blog.hotdry.top),
+ *    section 五 实践建议; "DeepSeek 开源周第二弹" (czhn.yksolo.com) (原生 FP8
  *    调度支持).
- *  - quantisation fused into the data movement: bjdmk.com.cn section 3.2.
+ *  - quantisation fused into the data movement: "DeepEP：专为MoE模型打造的
+ *    All-to-All通信库", section 3.2.
  *
  * Readings where the pages are silent (each one is a choice, stated here):
  *  - FP8 is OCP E4M3 ("fn": bias 7, 3 mantissa bits, no infinity, S.1111.111
@@ -224,7 +225,7 @@ int epo_layout_padded(int64_t T, int64_t k, int64_t E, int64_t R, int64_t M, con
 
 /* Group-limited gating: experts are split into groups and a token first
  * chooses groups, then experts inside them ("top-4 groups, top-8 experts":
- * blog.hotdry.top section 一 and section 三 on group-limited gating). */
+ * "deepep-expert-parallel-communication-library", section 一 and section 三 on group-limited gating). */
 int epo_route_group_limited(int64_t T, int64_t E, int64_t k, int64_t n_groups, int64_t topk_groups,
                             const float* scores, int64_t* topk_idx, float* topk_weights) {
   if (n_groups < 1 || E % n_groups != 0 || topk_groups < 1 || topk_groups > n_groups) return EPO_INVALID;

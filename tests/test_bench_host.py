@@ -94,3 +94,19 @@ def test_load_skew_is_max_over_mean_of_the_layout_counts():
     assert load["tokens_per_expert_max_over_mean"] == 6 / 2
     assert load["rows_per_rank_max_over_mean"] == round(12 / 8, 3)  # rank rows 12 and 4
     assert load["tokens_per_rank_max_over_mean"] == round(5 / 4, 3)
+
+
+def test_reshape_options():
+    """The profiling reshapes keep every other field of the workload."""
+    import argparse
+    base = dict(workload="decode", tokens_per_rank=0, dispatch_dtype="default", route=False, max_tokens_per_rank=0,
+                hidden=0, experts=0, groups=0, topk_groups=0, ranks=0)
+    w0 = bench.workload(argparse.Namespace(**base))
+    w = bench.workload(argparse.Namespace(**dict(base, ranks=16)))
+    assert (w.R, w.T, w.T // w.R) == (16, 2048, w0.T // w0.R) and w.E == w0.E and w.H == w0.H
+    w = bench.workload(argparse.Namespace(**dict(base, hidden=1024, tokens_per_rank=4096)))
+    assert (w.H, w.T, w.R) == (1024, 8 * 4096, 8) and w.use_fp8
+    w = bench.workload(argparse.Namespace(**dict(base, experts=160, groups=4, topk_groups=2)))
+    assert (w.E, w.n_groups, w.topk_groups, w.routing, w.k) == (160, 4, 2, "group", 8)
+    w = bench.workload(argparse.Namespace(**dict(base, groups=8, topk_groups=8)))
+    assert (w.E, w.n_groups, w.topk_groups) == (256, 8, 8)

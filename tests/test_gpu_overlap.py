@@ -1,8 +1,10 @@
 """SM budget and overlap with compute.
 
 The caller decides how many SMs the dispatch / combine kernels may fill, so
-that its own compute can run beside them (blog.hotdry.top, section 二, SM
-资源控制; the DeepEP guide's async / compute-stream options, zhouruolin.cn,
+that its own compute can run beside them
+("deepep-expert-parallel-communication-library", section 二 SM 资源控制; the
+DeepEP guide's async / compute-stream options, "DeepEP：MoE 专家并行 EP 通信
+kernel 编译与使用指南",
 section 五).  Here the whole path runs on a side stream with a small
 ``num_sms`` while a cuBLAS GEMM runs on the launching stream, the two ordered
 only by events.  Every output must be bit-identical to a plain run of the
