@@ -26,7 +26,9 @@ namespace ep {
 struct MoveParams {
   int T, H, k, G;
   int chunks;  // ceil(H / kChunk)
-  int pdl;     // 1: launched with programmatic dependent launch (the prologue prefetches)
+  int pdl;     // 1: launched with programmatic dependent launch: the kernel runs the
+               // prologue of common.cuh (allow the next kernel, prefetch, wait);
+               // 0: it skips it
   const int32_t* slot_of_pair;
   const float* topk_weights;
 };
@@ -122,8 +124,8 @@ dispatch_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__
                 float* __restrict__ recv_scale, float* __restrict__ recv_weight) {
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
-  pdl_allow_next();
-  pdl_wait_prev();
+  if (p.pdl) pdl_allow_next();
+  if (p.pdl) pdl_wait_prev();
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int t = static_cast<int>(u / p.chunks);
@@ -241,12 +243,10 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
 
   uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
   int t = blockIdx.x;
-  pdl_allow_next();
-  // the prefetch pays only while a previous kernel drains (at full batch it
-  // measured 3 % slower, the loads below following it at once)
-  if (p.pdl && t < p.T)
-    prefetch_l2(x + static_cast<int64_t>(t) * p.H, 2 * static_cast<int64_t>(p.H), threadIdx.x, blockDim.x);
-  pdl_wait_prev();
+  // no prefetch in this prologue: its code cost the kernel a register spill
+  // and 2-3 % at full batch
+  if (p.pdl) pdl_allow_next();
+  if (p.pdl) pdl_wait_prev();
   if (t < p.T) {
     const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
     if (a0) v0 = ld_ro_v4(xr + h0);
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kMoveThreads)
 gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __restrict__ out) {
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t nunits = static_cast<int64_t>(p.T) * p.chunks;
-  pdl_allow_next();
+  if (p.pdl) pdl_allow_next();
   {  // the first unit's slots (and weights) are this warp's first loads
     const int64_t u0 = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp;
     if (p.pdl && u0 < nunits && lane == 0) {
@@ -346,7 +346,7 @@ gather_reduce_kernel(MoveParams p, const uint16_t* __restrict__ y, uint16_t* __r
       if (WEIGHTED) prefetch_l2(p.topk_weights + pair0, 4 * p.k, 0, 1);
     }
   }
-  pdl_wait_prev();
+  if (p.pdl) pdl_wait_prev();
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < nunits;
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int t = static_cast<int>(u / p.chunks);
@@ -431,7 +431,7 @@ combine_backward_kernel(MoveParams p, const uint16_t* __restrict__ g, const uint
   const uint64_t evict_first = l2_evict_first_policy();
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t npairs = static_cast<int64_t>(p.T) * p.k;
-  pdl_allow_next();
+  if (p.pdl) pdl_allow_next();
   {  // the first pair's slot, weight and grad_out row are this warp's first loads
     const int64_t u0 = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp;
     if (p.pdl && u0 < npairs) {
@@ -444,7 +444,7 @@ combine_backward_kernel(MoveParams p, const uint16_t* __restrict__ g, const uint
         prefetch_l2(g + (u0 / p.k) * p.H, 2 * static_cast<int64_t>(p.H), lane, kWarp);
     }
   }
-  pdl_wait_prev();
+  if (p.pdl) pdl_wait_prev();
   for (int64_t u = static_cast<int64_t>(blockIdx.x) * kMoveWarps + threadIdx.x / kWarp; u < npairs;
        u += static_cast<int64_t>(gridDim.x) * kMoveWarps) {
     const int s = p.slot_of_pair[u];

@@ -187,3 +187,18 @@ def test_deterministic(cuda_device):
             assert np.array_equal(a, b)
         else:
             assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+
+
+@pytest.mark.parametrize("T,H,use_fp8,num_sms", [
+    (1024, 7040, True, 0),    # ragged last chunk (13.75 chunks)
+    (1024, 6656, True, 0),    # 13 chunks
+    (1024, 7168, False, 0),   # BF16 rows
+    (40, 7168, True, 4),      # SM budget: several tokens per CTA, the next one prefetched into registers
+    (60, 6656, False, 4),     # several tokens per CTA, the row stages reused
+])
+def test_small_batch_bulk_store_dispatch(cuda_device, T, H, use_fp8, num_sms):
+    """Small batches with 1536 < H <= 8192: the bulk-store dispatch on a
+    persistent grid, whole GPU or under an SM budget, against the oracle in
+    full."""
+    k, E, R = 8, 64, 4
+    run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=T + H), num_sms=num_sms)
