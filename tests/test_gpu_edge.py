@@ -202,3 +202,18 @@ def test_small_batch_bulk_store_dispatch(cuda_device, T, H, use_fp8, num_sms):
     full."""
     k, E, R = 8, 64, 4
     run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=T + H), num_sms=num_sms)
+
+
+@pytest.mark.parametrize("T,H,k,masked,num_sms", [
+    (96, 512, 6, 0.25, 0),     # masked and duplicate pairs, k < 8
+    (1024, 1024, 1, 0.0, 0),   # k = 1
+    (500, 2048, 8, 0.1, 3),    # SM budget: each warp strides over many units
+    (4, 512, 8, 0.0, 0),       # fewer units than warps
+])
+def test_small_batch_gathers(cuda_device, T, H, k, masked, num_sms):
+    """Small batches with k <= 8 and H a multiple of 512 (the persistent grid,
+    few units per warp or fewer units than warps): combine and dispatch
+    backward against the oracle in full."""
+    E, R = 32, 4
+    idx = random_idx(T, k, E, seed=T + k, masked=masked, distinct=masked == 0.0)
+    run_and_compare(cuda_device, T, H, k, E, R, False, idx, num_sms=num_sms)
