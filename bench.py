@@ -55,15 +55,16 @@ def call_bytes(w) -> dict:
     }
 
 
-# DRAM bytes per launch of the dominant kernel, from a full-size ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum; see profiles/).  An entry only
-# holds for the kernel sources and the launch configuration (the host file
-# picks the grids) it was taken on: if their hash differs, the bench reports
-# traffic as null.
+# DRAM bytes per launch of the dominant kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum), captured by ncu on the prefill shape cut to 512
+# tokens per rank and scaled to the full launch by the tokens processed (x8;
+# the counters grow with the tokens).  An entry only holds for the kernel
+# sources and the launch configuration (the host file picks the grids) it was
+# taken on: if their hash differs, the bench reports traffic as null.
 MEASURED_TRAFFIC = {
     ("prefill", 32768, "combine_backward"): {
-        "bytes": 4.23e9 + 3.70e9,
-        "sources_sha1": "7ac99dbbf5bc23a3907e7447e8d1c89ef869cc42",
+        "bytes": 8 * (528.779776e6 + 413.687552e6),
+        "sources_sha1": "2158a7258d4303b178c78c4fd12ab5104fc350b1",
     },
 }
 KERNEL_SOURCES = ("combine_ep_get_histogram_b200/csrc/common.cuh",
@@ -687,7 +688,8 @@ def run_ours(args, rank, world, local):
                      "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 3),
                      "peak_source": f"{peak_kind} hbm_gbs",
                      "bytes_per_launch": nb[dominant], "traffic": traffic,
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, full-size launch"},
+                     "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum at 512 tokens per rank, "
+                                        "scaled to the full launch by the tokens processed")},
         "clocks": clocks,
         "gpu_launches": (launches_per_step(w, args.peers) + (1 if args.route else 0)) * args.steps,
         "timing": ("CUDA graph replay of the step (the kernels alone; the per-call times come from a second graph "

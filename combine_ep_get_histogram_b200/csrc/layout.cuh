@@ -355,7 +355,11 @@ layout_small_kernel(LayoutParams p) {
   for (int i = threadIdx.x; i < ntok * p.R; i += blockDim.x) flags[i] = 0;
   __syncthreads();
 
-  // ---- phase 1: count this tile
+  // ---- phase 1: count this tile.  When the tile's tokens all belong to one
+  // source rank (the decode shape: one rank per CTA), its (rank, expert)
+  // counts are the tile's expert histogram and need no counting of their own.
+  const int r_first = ntok > 0 ? t0 / p.Tr : 0;
+  const bool one_rank = ntok > 0 && (t1 - 1) / p.Tr == r_first;
   int32_t* wh = whist + warp * p.E;
 #pragma unroll
   for (int q = 0; q < kSmallChunks; ++q) {
@@ -365,9 +369,11 @@ layout_small_kernel(LayoutParams p) {
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && lane == __ffs(same) - 1) wh[e] += __popc(same);
     const int tl = e >= 0 ? i / p.k : 0;  // token within the tile
-    const int key = e >= 0 ? ((t0 + tl) / p.Tr) * p.E + e : -1;
-    const unsigned same_key = __match_any_sync(0xffffffffu, key);
-    if (key >= 0 && lane == __ffs(same_key) - 1) atomicAdd(&cnt[key], __popc(same_key));
+    if (!one_rank) {
+      const int key = e >= 0 ? ((t0 + tl) / p.Tr) * p.E + e : -1;
+      const unsigned same_key = __match_any_sync(0xffffffffu, key);
+      if (key >= 0 && lane == __ffs(same_key) - 1) atomicAdd(&cnt[key], __popc(same_key));
+    }
     if (e >= 0) flags[tl * p.R + e / p.Er] = 1;
     __syncwarp();
   }
@@ -376,6 +382,7 @@ layout_small_kernel(LayoutParams p) {
     int32_t tot = 0;
     for (int w = 0; w < kSmallWarps; ++w) tot += whist[w * p.E + e];
     hist[e] = tot;
+    if (one_rank) cnt[r_first * p.E + e] = tot;
   }
   for (int b0 = 0; b0 < ntok * p.R; b0 += blockDim.x) {  // uniform trip count
     const int i = b0 + threadIdx.x;

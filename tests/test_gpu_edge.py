@@ -124,6 +124,8 @@ def test_empty_input(cuda_device):
     (256, 8704, 4, 64, 8, False),      # past the TMA width: warp dispatch
     (300, 1024, 3, 16, 4, False),      # k = 3 with H % 512 = 0: a gather batch with unused row slots
     (256, 1536, 12, 48, 8, True),      # k = 12: a gather batch of 8 rows and one of 4
+    (99, 256, 4, 48, 3, False),        # one-CTA layout tiles that straddle two source ranks
+    (1024, 512, 8, 128, 16, True),     # every one-CTA layout tile holds two source ranks
 ])
 def test_shapes(cuda_device, T, H, k, E, R, use_fp8):
     run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=T + k))
