@@ -54,7 +54,11 @@
  *    when the environment variable EP_DEBUG=1 is set).
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream).  Calls on one handle must not overlap; results are defined
- *    once the stream reaches them.
+ *    once the stream reaches them.  Below 16 tokens per SM the kernels are
+ *    launched with programmatic dependent launch (EP_PDL=0 turns it off): a
+ *    kernel may become resident while the previous kernel on the stream
+ *    finishes, but it reads and writes no global memory before that kernel
+ *    has completed, so stream order is kept for any predecessor.
  *  - bf16 arrays are uint16 bit patterns; rows of bf16 / fp8 arrays must start
  *    on 16-byte boundaries (H % 8 == 0 and 16-byte aligned base pointers).
  *  - Return value: EP_OK or an ep_status_t code.  Argument errors are found
