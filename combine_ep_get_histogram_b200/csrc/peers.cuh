@@ -204,16 +204,10 @@ dispatch_tma_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows
       if (a0) n0 = ld_ro_v4(xr + h0);
       if (a1) n1 = ld_ro_v4(xr + h1);
     }
-    // the row stage is free once the copies issued L.stages tokens ago have read it
+    // the row stage is free once the copies issued L.stages tokens ago have
+    // read it (the first token's stage has had no copies)
     if (threadIdx.x == 0) bulk_wait_read_all_but(L.stages - 1);
-    if (warp == 0 && lane < p.k) {
-      int o, r;
-      peer_pair(p, row0, t, lane, o, r);
-      srow[lane] = r;
-      sowner[lane] = o;
-      sw[lane] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
-    }
-    __syncthreads();
+    if (it > 0) __syncthreads();
 
     if constexpr (FP8) {
       float sc0, sc1;
@@ -231,6 +225,15 @@ dispatch_tma_peers_kernel(PeerParams p, const uint16_t* __restrict__ x, PeerRows
     } else {
       if (a0) *reinterpret_cast<uint4*>(row + 2 * h0) = v0;
       if (a1) *reinterpret_cast<uint4*>(row + 2 * h1) = v1;
+    }
+    // the pairs' owners, rows and weights after the quantisation, as in
+    // dispatch_tma_kernel
+    if (warp == 0 && lane < p.k) {
+      int o, r;
+      peer_pair(p, row0, t, lane, o, r);
+      srow[lane] = r;
+      sowner[lane] = o;
+      sw[lane] = p.topk_weights[static_cast<int64_t>(t) * p.k + lane];
     }
     // make the generic-proxy shared-memory writes visible to the bulk copies
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -50,7 +50,10 @@ class PeerBuffers:
     the C ABI).
 
     Collective over `group` (a torch.distributed group, gloo is enough): every
-    rank passes buffers under the same names.  One all-gather of the
+    rank passes buffers under the same names.  The buffers must live in
+    cudaMalloc allocations (torch's default caching allocator; not its
+    expandable segments, whose memory CUDA IPC cannot export: the export
+    raises).  One all-gather of the
     80-byte export records, then each rank maps the others' buffers.
     ``table(name)`` lists the device addresses in rank order, this rank's own
     entry being its local pointer.  ``close()`` unmaps every buffer this rank
