@@ -152,3 +152,17 @@ def test_route_bad_arguments_rejected_on_host(ng, tg, k):
     s = ep.make_shape(T=64, H=128, k=k, E=64, R=4)
     fake = 1 << 20
     assert ep.library().ep_route_group_limited(ctypes.byref(s), fake, ng, tg, fake, fake, None) == 1
+
+
+def test_ipc_calls_reject_bad_arguments_on_host():
+    """The CUDA-IPC helpers check their pointers before any CUDA call."""
+    lib = ep.library()
+    rec = binding.ep_ipc_buffer_t()
+    base, ptr = ctypes.c_void_p(), ctypes.c_void_p()
+    assert ctypes.sizeof(rec) == 80
+    assert lib.ep_ipc_export(None, ctypes.byref(rec)) == binding.EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_export(4096, None) == binding.EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_open(None, ctypes.byref(base), ctypes.byref(ptr)) == binding.EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_open(ctypes.byref(rec), None, ctypes.byref(ptr)) == binding.EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_open(ctypes.byref(rec), ctypes.byref(base), None) == binding.EP_ERR_INVALID_ARG
+    assert lib.ep_ipc_close(None) == binding.EP_ERR_INVALID_ARG
