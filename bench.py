@@ -64,7 +64,7 @@ def call_bytes(w) -> dict:
 MEASURED_TRAFFIC = {
     ("prefill", 32768, "combine_backward"): {
         "bytes": 8 * (528.778240e6 + 413.370880e6),
-        "sources_sha1": "c9c7c8655816a63dd0465e57ea4b92a99641a07e",
+        "sources_sha1": "866db7c78f2bb2b42d524c42c2abff8b37b4ec98",
     },
 }
 KERNEL_SOURCES = ("combine_ep_get_histogram_b200/csrc/common.cuh",
@@ -73,14 +73,14 @@ KERNEL_SOURCES = ("combine_ep_get_histogram_b200/csrc/common.cuh",
 
 
 def code_lines(text: str) -> str:
-    """The source without // comments, trailing blanks and blank lines, so
-    that a comment edit leaves the hash of the code unchanged."""
-    out = []
-    for line in text.splitlines():
-        code = line.split("//", 1)[0].rstrip()
-        if code:
-            out.append(code)
-    return "\n".join(out)
+    """The source's tokens without // comments and without the layout between
+    them: whitespace is kept only where it separates two identifier or number
+    characters.  A comment edit or a rewrapped line leaves the hash of the
+    code unchanged."""
+    import re
+    code = " ".join(line.split("//", 1)[0] for line in text.splitlines())
+    code = re.sub(r"\s+", " ", code)
+    return re.sub(r"(?<=\W) | (?=\W)", "", code).strip()
 
 
 def kernel_sources_sha1(read=None) -> str:

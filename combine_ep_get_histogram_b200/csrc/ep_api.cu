@@ -501,7 +501,8 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
     return finish(handle, s);
   }
   if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
-    launch(pdl, layout_small_kernel, kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R), s, p);
+    launch(pdl, layout_small_kernel, kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R),
+        s, p);
     return finish(handle, s);
   }
   if (g.nt > 0) {
@@ -545,11 +546,11 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
     }
     const int grid = tma_dispatch_grid(*d, shape, T, occ);
     if (fp8)
-      launch(pdl, dispatch_tma_kernel<true>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x, recv_scale,
-          recv_weight);
+      launch(pdl, dispatch_tma_kernel<true>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x,
+          recv_scale, recv_weight);
     else
-      launch(pdl, dispatch_tma_kernel<false>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x, nullptr,
-          recv_weight);
+      launch(pdl, dispatch_tma_kernel<false>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x,
+          nullptr, recv_weight);
   } else if (shape->use_fp8) {
     launch(pdl, dispatch_kernel<true>, movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s, p,
         static_cast<const uint16_t*>(x), recv_x, recv_scale, recv_weight);
@@ -605,9 +606,11 @@ int ep_combine_backward(const ep_shape_t* shape, const void* grad_out, const voi
   const uint16_t* gp = static_cast<const uint16_t*>(grad_out);
   const uint16_t* yp = static_cast<const uint16_t*>(y);
   if (ragged)
-    launch(pdl, combine_backward_kernel<true>, grid, kMoveThreads, 0, s, p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
+    launch(pdl, combine_backward_kernel<true>, grid, kMoveThreads, 0, s, p, gp, yp, static_cast<uint16_t*>(grad_y),
+        grad_w);
   else
-    launch(pdl, combine_backward_kernel<false>, grid, kMoveThreads, 0, s, p, gp, yp, static_cast<uint16_t*>(grad_y), grad_w);
+    launch(pdl, combine_backward_kernel<false>, grid, kMoveThreads, 0, s, p, gp, yp, static_cast<uint16_t*>(grad_y),
+        grad_w);
   return finish(handle, s);
 }
 
@@ -627,11 +630,11 @@ int ep_dispatch_backward(const ep_shape_t* shape, const void* grad_recv, const e
   const bool ragged = shape->H % kChunk != 0;
   const int grid = movement_grid(*d, shape, d->occ_dbwd[ragged], T * p.chunks);
   if (ragged)
-    launch(pdl, gather_reduce_kernel<false, true>, grid, kMoveThreads, 0, s, p, static_cast<const uint16_t*>(grad_recv),
-        static_cast<uint16_t*>(grad_x));
+    launch(pdl, gather_reduce_kernel<false, true>, grid, kMoveThreads, 0, s, p,
+        static_cast<const uint16_t*>(grad_recv), static_cast<uint16_t*>(grad_x));
   else
-    launch(pdl, gather_reduce_kernel<false, false>, grid, kMoveThreads, 0, s, p, static_cast<const uint16_t*>(grad_recv),
-        static_cast<uint16_t*>(grad_x));
+    launch(pdl, gather_reduce_kernel<false, false>, grid, kMoveThreads, 0, s, p,
+        static_cast<const uint16_t*>(grad_recv), static_cast<uint16_t*>(grad_x));
   return finish(handle, s);
 }
 
@@ -751,11 +754,11 @@ int ep_dispatch_peers(const ep_shape_t* shape, int32_t rank, const int64_t* topk
     else
       launch(pdl, dispatch_tma_peers_kernel<false>, grid, threads, smem, s, p, xs, rx, rs, rw);
   } else if (fp8) {
-    launch(pdl, dispatch_peers_kernel<true>, movement_grid(*d, shape, d->occ_peer_disp[1], units), kMoveThreads, 0, s, p, xs,
-        rx, rs, rw);
+    launch(pdl, dispatch_peers_kernel<true>, movement_grid(*d, shape, d->occ_peer_disp[1], units), kMoveThreads, 0,
+        s, p, xs, rx, rs, rw);
   } else {
-    launch(pdl, dispatch_peers_kernel<false>, movement_grid(*d, shape, d->occ_peer_disp[0], units), kMoveThreads, 0, s, p,
-        xs, rx, rs, rw);
+    launch(pdl, dispatch_peers_kernel<false>, movement_grid(*d, shape, d->occ_peer_disp[0], units), kMoveThreads, 0,
+        s, p, xs, rx, rs, rw);
   }
   return finish(handle, s);
 }

@@ -1,5 +1,6 @@
 """Host-side helpers of bench.py that need no GPU: the code hash that keeps a
-measured DRAM-traffic figure tied to the kernel it was taken on, and the L2
+measured DRAM-traffic figure tied to the kernel it was taken on (comments
+and layout whitespace aside), and the L2
 statement made from a step's bytes."""
 
 import os
@@ -20,6 +21,19 @@ def test_comment_edits_keep_the_code_hash():
     assert base == bench.kernel_sources_sha1()
     commented = bench.kernel_sources_sha1(_reader(lambda f, t: t.replace("\n", "  // note\n\n", 3) + "// end\n"))
     assert commented == base
+
+
+def test_rewrapped_lines_keep_the_code_hash():
+    base = bench.kernel_sources_sha1()
+
+    def rewrap(f, t):
+        out = []
+        for line in t.splitlines():
+            code, sep, comment = line.partition("//")
+            out.append(code.replace(", ", ",\n      ").replace("    ", "\t") + sep + comment)
+        return "\n".join(out)
+
+    assert bench.kernel_sources_sha1(_reader(rewrap)) == base
 
 
 def test_code_edits_change_the_code_hash():
