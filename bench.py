@@ -482,6 +482,7 @@ def run_ours(args, rank, world, local):
     # the per-call breakdown (event nodes between two kernels add their own
     # latency and keep a kernel from starting while the previous one drains).
     per_call_ms = {c: [] for c in calls}
+    same_size_copy_us = None
     if args.no_graph:
         run_step = path.step
     else:
@@ -530,6 +531,38 @@ def run_ours(args, rank, world, local):
             torch.cuda.synchronize()
             for ci, c in enumerate(calls):
                 per_call_ms[c].append(call_ms(cmarks, ci, True))
+        # the same method around a device-to-device copy (cudaMemcpyAsync)
+        # that moves each call's bytes (half read, half written): what a
+        # plain copy of that size reaches when it is timed this way
+        half = {c: max(16, nb[c] // 2 // 16 * 16) for c in calls}
+        csrc = torch.ones(max(half.values()), dtype=torch.uint8, device=dev)
+        cdst = torch.empty_like(csrc)
+        kmarks = [torch.cuda.Event(enable_timing=True, external=not args.no_graph) for _ in range(2 * len(calls))]
+
+        def copies_once():
+            for ci, c in enumerate(calls):
+                cold_flush()
+                kmarks[2 * ci].record()
+                cdst[:half[c]].copy_(csrc[:half[c]])
+                kmarks[2 * ci + 1].record()
+
+        if args.no_graph:
+            run_copies = copies_once
+        else:
+            copy_graph = torch.cuda.CUDAGraph()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(copy_graph):
+                copies_once()
+            run_copies = copy_graph.replay
+        copy_ms = {c: [] for c in calls}
+        for i in range(2 + min(args.steps, 20)):
+            run_copies()
+            torch.cuda.synchronize()
+            if i >= 2:
+                for ci, c in enumerate(calls):
+                    copy_ms[c].append(kmarks[2 * ci].elapsed_time(kmarks[2 * ci + 1]))
+        same_size_copy_us = {c: 1e3 * statistics.median(v) for c, v in copy_ms.items()}
+        del csrc, cdst
         barrier()
 
     # device-timed region: K steps back to back on the launching stream
@@ -656,6 +689,10 @@ def run_ours(args, rank, world, local):
         per_call[c] = {"us": round(us, 2), "us_median": round(1e3 * statistics.median(per_call_ms[c]), 2),
                        "bytes": nb[c], "GB_s": round(nb[c] / (us * 1e-6) / 1e9, 1),
                        "frac_of_peak": round(nb[c] / (us * 1e-6) / 1e9 / peak, 3)}
+        if same_size_copy_us is not None:
+            cu = same_size_copy_us[c]
+            per_call[c]["same_size_copy"] = {"us": round(cu, 2), "GB_s": round(nb[c] / (cu * 1e-6) / 1e9, 1),
+                                             "frac_of_copy": round(cu / us, 3)}
     dominant = max((c for c in calls), key=lambda c: per_call[c]["us"])
     kernel_of = {"dispatch": "dispatch_tma_kernel<FP8>" if w.use_fp8 else "dispatch_tma_kernel<BF16>",
                  "combine": "gather_reduce_kernel<weighted>", "combine_backward": "combine_backward_kernel",
