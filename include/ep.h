@@ -66,7 +66,8 @@
  *    found on the device: the pair is treated as masked and bit 0 of
  *    handle->error_word is set; ep_get_error reports it.
  *  - Limits: 0 <= T, T % R == 0, 1 <= k <= 32, 1 <= E <= 1024, 1 <= R <= E,
- *    E % R == 0, T*k < 2^31, 8 <= H, H % 8 == 0 (H % 128 == 0 with FP8);
+ *    R <= 256, E % R == 0, T*k < 2^31, 8 <= H, H % 8 == 0 (H % 128 == 0 with
+ *    FP8), use_fp8 0 or 1, num_sms >= 0;
  *    padded layout: see max_tokens_per_rank.
  */
 #ifndef EP_B200_H

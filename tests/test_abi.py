@@ -61,6 +61,8 @@ BAD_SHAPES = [
     dict(T=64, H=250, k=4, E=16, R=4),      # H % 8
     dict(T=64, H=320, k=4, E=16, R=4, use_fp8=True),  # H % 128 with FP8
     dict(T=64, H=256, k=4, E=4, R=8),       # R > E
+    dict(T=512, H=256, k=4, E=512, R=512),  # R > 256
+    dict(T=1 << 28, H=256, k=8, E=16, R=4),  # T * k >= 2^31
     dict(T=-4, H=256, k=4, E=16, R=4),
     dict(T=64, H=256, k=4, E=16, R=4, num_sms=-1),
 ]
@@ -78,6 +80,11 @@ def test_bad_shapes_rejected_on_host(kw):
     assert lib.ep_combine(ctypes.byref(s), fake, fake, ctypes.byref(h), fake, None) == 1
     assert lib.ep_combine_backward(ctypes.byref(s), fake, fake, fake, ctypes.byref(h), fake, fake, None) == 1
     assert lib.ep_dispatch_backward(ctypes.byref(s), fake, ctypes.byref(h), fake, None) == 1
+
+
+def test_use_fp8_must_be_zero_or_one():
+    s = binding.ep_shape_t(64, 256, 4, 16, 4, 2, 0, 0)  # make_shape would coerce it to 1
+    assert ep.library().ep_workspace_size(ctypes.byref(s)) == 0
 
 
 def test_bad_pointers_rejected_on_host():

@@ -126,6 +126,8 @@ def test_empty_input(cuda_device):
     (256, 1536, 12, 48, 8, True),      # k = 12: a gather batch of 8 rows and one of 4
     (99, 256, 4, 48, 3, False),        # one-CTA layout tiles that straddle two source ranks
     (1024, 512, 8, 128, 16, True),     # every one-CTA layout tile holds two source ranks
+    (512, 256, 8, 256, 256, False),    # R at its maximum, one expert per rank, 2 tokens per rank
+    (256 * 40, 128, 4, 1024, 256, True),  # R and E at their maxima, tiled layout
 ])
 def test_shapes(cuda_device, T, H, k, E, R, use_fp8):
     run_and_compare(cuda_device, T, H, k, E, R, use_fp8, random_idx(T, k, E, seed=T + k))

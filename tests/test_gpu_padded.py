@@ -86,6 +86,12 @@ def test_padded_rank_counts(cuda_device, R):
     run_padded(cuda_device, T, H, k, E, R, T // R + 2, R % 2 == 1, routing(T, k, E, seed=R, masked=0.1))
 
 
+def test_padded_max_ranks(cuda_device):
+    """R = 256 ranks (the maximum), one expert per rank, 2 tokens per rank."""
+    T, H, k, E, R = 512, 256, 4, 256, 256
+    run_padded(cuda_device, T, H, k, E, R, T // R + 2, False, routing(T, k, E, seed=11, masked=0.1))
+
+
 def test_padded_capacity_overflow_masked_and_bad(cuda_device):
     T, H, k, E, R = 64, 256, 4, 8, 4
     idx = routing(T, k, E, seed=3, masked=0.2, duplicates=True)
