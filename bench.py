@@ -38,6 +38,8 @@ if ROOT not in sys.path:
 METRIC = "dispatch/combine µs/call & effective HBM GB/s vs B200 roofline, 1 GPU"
 CALLS = ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward")
 ROUTE_CALLS = ("route",) + CALLS
+# --fused-dispatch: the layout and the dispatch as one call (ep_dispatch_with_layout)
+FUSED_CALLS = ("dispatch_with_layout", "combine", "combine_backward", "dispatch_backward")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -52,6 +54,7 @@ def call_bytes(w) -> dict:
         "combine": T * k * H * 2 + T * k * 4 + T * H * 2,
         "combine_backward": T * H * 2 + 2 * T * k * H * 2 + 2 * T * k * 4,
         "dispatch_backward": T * k * H * 2 + T * H * 2,
+        "dispatch_with_layout": T * k * 8 + T * R + 2 * T * k * 4 + disp,
     }
 
 
@@ -63,8 +66,8 @@ def call_bytes(w) -> dict:
 # taken on: if their hash differs, the bench reports traffic as null.
 MEASURED_TRAFFIC = {
     ("prefill", 32768, "combine_backward"): {
-        "bytes": 8 * (528.778240e6 + 413.370880e6),
-        "sources_sha1": "866db7c78f2bb2b42d524c42c2abff8b37b4ec98",
+        "bytes": 8 * (528.872960e6 + 415.468544e6),
+        "sources_sha1": "4650901c1339a4c060cbfa701c296a7511a363dd",
     },
 }
 KERNEL_SOURCES = ("combine_ep_get_histogram_b200/csrc/common.cuh",
@@ -239,7 +242,7 @@ def call_ms(marks, ci: int, cold: bool) -> float:
 class Path:
     """Device buffers of one workload and one step through the C ABI."""
 
-    def __init__(self, w, d, dev, max_tokens_per_rank=0, route=False, num_sms=0):
+    def __init__(self, w, d, dev, max_tokens_per_rank=0, route=False, num_sms=0, fused=False):
         import numpy as np
         import torch
         import combine_ep_get_histogram_b200 as ep
@@ -253,6 +256,7 @@ class Path:
         self.host = {"topk_idx": torch.from_numpy(d["topk_idx"]), "topk_weights": torch.from_numpy(d["topk_weights"]),
                      "x": bf16(d["x"]), "y": bf16(d["y"]), "g": bf16(d["g"])}
         self.route = route
+        self.fused = fused
         if route:
             self.host["scores"] = torch.from_numpy(d["scores"])
         self.inp = {n: t.to(dev) for n, t in self.host.items()}
@@ -278,13 +282,19 @@ class Path:
             ep.ep_route_group_limited(self.shape, i["scores"], self.w.n_groups, self.w.topk_groups, i["topk_idx"],
                                       i["topk_weights"])
             m.end()
-        m.begin()
-        ep.ep_get_dispatch_layout(self.shape, i["topk_idx"], self.handle, self.ws)
-        m.end()
-        m.begin()
-        ep.ep_dispatch(self.shape, i["x"], i["topk_weights"], self.handle, self.recv_x, self.recv_scale,
-                       self.recv_weight)
-        m.end()
+        if self.fused:
+            m.begin()
+            ep.ep_dispatch_with_layout(self.shape, i["topk_idx"], i["x"], i["topk_weights"], self.handle, self.ws,
+                                       self.recv_x, self.recv_scale, self.recv_weight)
+            m.end()
+        else:
+            m.begin()
+            ep.ep_get_dispatch_layout(self.shape, i["topk_idx"], self.handle, self.ws)
+            m.end()
+            m.begin()
+            ep.ep_dispatch(self.shape, i["x"], i["topk_weights"], self.handle, self.recv_x, self.recv_scale,
+                           self.recv_weight)
+            m.end()
         if before_back is not None:
             before_back()
         m.begin()
@@ -394,7 +404,7 @@ def l2_policy(step_bytes: int, l2_bytes: int) -> tuple:
                   f"{2 * l2_bytes / 2**20:.0f} MiB read, outside the timed region; each step timed on its own)")
 
 
-MOVEMENT_CALLS = ("dispatch", "combine", "combine_backward", "dispatch_backward")
+MOVEMENT_CALLS = ("dispatch", "dispatch_with_layout", "combine", "combine_backward", "dispatch_backward")
 
 
 def per_call_policy(nb: dict, l2_bytes: int) -> tuple:
@@ -428,7 +438,9 @@ def bench_config(w, args, world: int, l2_bytes: int = B200_L2_BYTES) -> dict:
             "parallelism": (f"replicas x{world}" if world > 1 else
                             f"1 GPU, {w.R} ranks emulated through the peer-table calls"
                             if getattr(args, "peers", False) else "1 GPU, virtual ranks"),
-            "router_in_step": bool(args.route)}
+            "router_in_step": bool(args.route),
+            "dispatch_call": ("fused: ep_dispatch_with_layout" if getattr(args, "fused_dispatch", False)
+                              else "separate: ep_get_dispatch_layout, then ep_dispatch")}
 
 
 def run_ours(args, rank, world, local):
@@ -445,9 +457,9 @@ def run_ours(args, rank, world, local):
     d = wl.make_inputs(w, parts=("routing", "x", "g") + (() if M else ("y",)) + (("scores",) if args.route else ()))
     if M:  # expert outputs fill the padded receive rows
         d["y"] = wl.normal_bf16(w.E * w.R * M, w.H, w.seed, 2)
-    if args.peers and (M or args.route):
-        raise SystemExit("--peers runs the dense layout without routing")
-    path = PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route)
+    if args.peers and (M or args.route or args.fused_dispatch):
+        raise SystemExit("--peers runs the dense layout and separate calls, without routing")
+    path = PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route, fused=args.fused_dispatch)
     nb = {c: v for c, v in call_bytes(w).items() if c in calls}
     step_bytes = sum(nb.values())
     nmarks = len(calls) + 1
@@ -606,7 +618,8 @@ def run_ours(args, rank, world, local):
     # third stream; PCIe is full duplex).
     e2e = None
     if not args.no_e2e:
-        paths = [path, PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route)]
+        paths = [path, PeersPath(w, d, dev) if args.peers else Path(w, d, dev, M, route=args.route,
+                                                                    fused=args.fused_dispatch)]
         pin = {n: t.pin_memory() for n, t in path.host.items()}
         outs = {"out": torch.empty_like(path.out, device="cpu").pin_memory(),
                 "grad_x": torch.empty_like(path.grad_x, device="cpu").pin_memory(),
@@ -697,6 +710,7 @@ def run_ours(args, rank, world, local):
     kernel_of = {"dispatch": "dispatch_tma_kernel<FP8>" if w.use_fp8 else "dispatch_tma_kernel<BF16>",
                  "combine": "gather_reduce_kernel<weighted>", "combine_backward": "combine_backward_kernel",
                  "dispatch_backward": "gather_reduce_kernel<unweighted>", "layout": "layout_*_kernel",
+                 "dispatch_with_layout": "layout_*_kernel + dispatch_tma_kernel (early form below 16 tokens per SM)",
                  "route": "route_compact_kernel|route_aligned_kernel|route_group_limited_kernel"}
     if args.peers:
         kernel_of.update({"dispatch": "dispatch_tma_peers_kernel" if 4 <= -(-w.H // 512) <= 16
@@ -771,8 +785,8 @@ def measure_overlap(args, w, d, dev, M, step_ms):
     on all SMs, then the path on all SMs.  The GEMM repeats are sized to
     about one full-GPU step of the path."""
     import torch
-    budget = Path(w, d, dev, M, route=args.route, num_sms=args.overlap_sms)
-    full = Path(w, d, dev, M, route=args.route)
+    budget = Path(w, d, dev, M, route=args.route, num_sms=args.overlap_sms, fused=args.fused_dispatch)
+    full = Path(w, d, dev, M, route=args.route, fused=args.fused_dispatch)
     n = 8192
     gen = torch.Generator(device=dev).manual_seed(0)
     a = torch.randn((n, n), device=dev, dtype=torch.bfloat16, generator=gen)
@@ -853,7 +867,8 @@ def workload(args):
 # -------------------------------------------------------- CPU oracle arm
 
 def step_calls(args) -> tuple:
-    return ROUTE_CALLS if args.route else CALLS
+    calls = FUSED_CALLS if getattr(args, "fused_dispatch", False) else CALLS
+    return (("route",) + calls) if args.route else calls
 
 
 def oracle_pass(w, d, route: bool, M: int):
@@ -966,6 +981,8 @@ def main():
     ap.add_argument("--groups", type=int, default=0, help="reshape: expert groups of the group-limited routing")
     ap.add_argument("--topk-groups", type=int, default=0, help="reshape: groups each token picks")
     ap.add_argument("--ranks", type=int, default=0, help="reshape: virtual ranks R (same tokens per rank)")
+    ap.add_argument("--fused-dispatch", action="store_true",
+                    help="the layout and the dispatch as one call (ep_dispatch_with_layout)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch each call eagerly instead of replaying a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")

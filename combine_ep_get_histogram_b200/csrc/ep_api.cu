@@ -44,7 +44,7 @@ struct DeviceInfo {
   int occ_count = 0, occ_scan = 0, occ_assign = 0;
   int occ_disp_bf16 = 0, occ_disp_fp8 = 0;
   int occ_comb[2] = {}, occ_dbwd[2] = {};  // [ragged]
-  int occ_tma[2][kTmaMaxChunks + 1] = {};  // [fp8][chunks], filled on first use
+  int occ_tma[2][2][kTmaMaxChunks + 1] = {};  // [early][fp8][chunks], filled on first use
   int occ_tma_peers[2][kTmaMaxChunks + 1] = {};  // the same for dispatch_tma_peers_kernel
   int occ_cbwd[2] = {};  // [ragged]
   int occ_peer_disp[2] = {}, occ_peer_gather[2][2] = {}, occ_peer_cbwd[2] = {};  // [fp8], [weighted][ragged], [ragged]
@@ -399,6 +399,139 @@ int peer_setup(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, c
   return EP_OK;
 }
 
+// The layout kernels of one call, enqueued on s (arguments checked by the
+// caller).  late: the last kernel lets the next one be scheduled only after
+// its own programmatic-launch wait (LayoutParams::late_trigger).
+int enqueue_layout(const ep_shape_t* shape, const int64_t* topk_idx, const ep_handle_t* handle, void* workspace,
+                   const LayoutGeometry& g, bool pdl, bool late, cudaStream_t s) {
+  int st = EP_OK;
+  LayoutParams p;
+  p.topk_idx = topk_idx;
+  p.T = shape->T;
+  p.k = shape->k;
+  p.E = shape->E;
+  p.R = shape->R;
+  p.Tr = shape->T / shape->R;
+  p.Er = shape->E / shape->R;
+  p.tile_t = g.tile_t;
+  p.tiles_per_rank = g.tiles_per_rank;
+  p.nt = g.nt;
+  p.ncol = g.ncol;
+  p.colhist = static_cast<int32_t*>(workspace);
+  p.coltotal = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + g.colhist_bytes);
+  p.num_tokens_per_expert = handle->num_tokens_per_expert;
+  p.expert_offset = handle->expert_offset;
+  p.num_tokens_per_rank = handle->num_tokens_per_rank;
+  p.count_src_rank_expert = handle->count_src_rank_expert;
+  p.src_rank_expert_offset = handle->src_rank_expert_offset;
+  p.is_token_in_rank = handle->is_token_in_rank;
+  p.slot_of_pair = handle->slot_of_pair;
+  p.src_of_slot = handle->src_of_slot;
+  p.error_word = handle->error_word;
+  p.late_trigger = late ? 1 : 0;
+
+  if (shape->max_tokens_per_rank > 0) {
+    const size_t smem = layout_padded_smem(p.Tr, shape->E, shape->R);
+    if (smem > 48 * 1024) {
+      // a function attribute belongs to the current context (a reset or a
+      // green context starts without it), so it is set before each launch
+      const void* fn = shape->R <= kPadClusterMax ? reinterpret_cast<const void*>(layout_padded_kernel<true>)
+                                                  : reinterpret_cast<const void*>(layout_padded_kernel<false>);
+      if ((st = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem)))) != EP_OK)
+        return st;
+    }
+    if (shape->R <= kPadClusterMax) {  // one cluster of R CTAs sums the totals itself
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(shape->R);
+      cfg.blockDim = dim3(kPadThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = shape->R;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = pdl_attribute(attr, 1, pdl);
+      return cuda_status(cudaLaunchKernelEx(&cfg, layout_padded_kernel<true>, p, shape->max_tokens_per_rank));
+    }
+    if ((st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_expert, 0, shape->E * 4, s))) != EP_OK ||
+        (st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_rank, 0, shape->R * 4, s))) != EP_OK)
+      return st;
+    launch(pdl, layout_padded_kernel<false>, shape->R, kPadThreads, smem, s, p, shape->max_tokens_per_rank);
+    return EP_OK;
+  }
+  if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
+    launch(pdl, layout_small_kernel, kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R),
+        s, p);
+    return EP_OK;
+  }
+  // only the last of the three kernels triggers late
+  LayoutParams pe = p;
+  pe.late_trigger = 0;
+  if (g.nt > 0) {
+    const size_t smem = static_cast<size_t>(g.ncol) * 4 + static_cast<size_t>(g.tile_t) * shape->R;
+    launch(pdl, layout_count_kernel, g.nt, kLayoutThreads, smem, s, pe);
+  }
+  launch(pdl, layout_scan_kernel, g.ncol, kLayoutThreads, 0, s, pe);
+  const size_t smem_assign = static_cast<size_t>(shape->E + 1 + kLayoutWarps * shape->E) * 4;
+  launch(pdl, layout_assign_kernel, g.nt > 0 ? g.nt : 1, kLayoutThreads, smem_assign, s, p);
+  return EP_OK;
+}
+
+// Argument checks of ep_dispatch.
+int check_dispatch_args(const ep_shape_t* shape, const void* x, const float* topk_weights, const ep_handle_t* handle,
+                        const void* recv_x, const float* recv_scale, const float* recv_weight) {
+  int st = check_shape(shape);
+  if (st != EP_OK) return st;
+  if ((st = check_handle(shape, handle)) != EP_OK) return st;
+  const int64_t T = shape->T, P = T * shape->k;
+  if (!rows_ok(x, T) || !rows_ok(recv_x, P) || !f32_ok(topk_weights, P)) return EP_ERR_INVALID_ARG;
+  if (shape->use_fp8 && !f32_ok(recv_scale, P)) return EP_ERR_INVALID_ARG;
+  if (recv_weight != nullptr && !aligned(recv_weight, 4)) return EP_ERR_INVALID_ARG;
+  return EP_OK;
+}
+
+// The bulk-store dispatch serves 4 to 16 chunks of 512 channels.
+bool tma_dispatch_applies(const ep_shape_t* shape) {
+  const int64_t chunks = ceil_div(shape->H, kChunk);
+  return chunks >= kTmaMinChunks && chunks <= kTmaMaxChunks;
+}
+
+// The dispatch kernel of one call (arguments checked, T > 0).  early: the
+// bulk-store kernel's EARLY form, only right after the fused call's layout.
+void enqueue_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weights, const ep_handle_t* handle,
+                      void* recv_x, float* recv_scale, float* recv_weight, const DeviceInfo* d, bool pdl, bool early,
+                      cudaStream_t s) {
+  const MoveParams p = move_params(shape, handle, topk_weights, pdl);
+  const int64_t units = shape->T * p.chunks;
+  const uint16_t* xp = static_cast<const uint16_t*>(x);
+  const bool fp8 = shape->use_fp8 != 0;
+  if (tma_dispatch_applies(shape)) {
+    const int threads = p.chunks * kWarp;
+    const size_t smem = tma_smem_layout(shape->H, fp8, early).total;
+    void (*fn)(MoveParams, const uint16_t*, void*, float*, float*) =
+        fp8 ? (early ? dispatch_tma_kernel<true, true> : dispatch_tma_kernel<true, false>)
+            : (early ? dispatch_tma_kernel<false, true> : dispatch_tma_kernel<false, false>);
+    int occ;
+    {
+      std::lock_guard<std::mutex> lock(g_dev_mu);
+      int& cached = const_cast<DeviceInfo*>(d)->occ_tma[early][fp8][p.chunks];
+      if (cached == 0) cached = occupancy(reinterpret_cast<const void*>(fn), threads, smem);
+      occ = cached;
+    }
+    const int grid = tma_dispatch_grid(*d, shape, shape->T, occ);
+    launch(pdl, fn, grid, threads, smem, s, p, xp, recv_x, fp8 ? recv_scale : nullptr, recv_weight);
+  } else if (fp8) {
+    launch(pdl, dispatch_kernel<true>, movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s, p, xp,
+        recv_x, recv_scale, recv_weight);
+  } else {
+    launch(pdl, dispatch_kernel<false>, movement_grid(*d, shape, d->occ_disp_bf16, units), kMoveThreads, 0, s, p, xp,
+        recv_x, nullptr, recv_weight);
+  }
+}
+
 }  // namespace
 
 // Argument checks of ep_get_dispatch_layout other than the workspace, shared
@@ -438,126 +571,44 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
     return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
-  const bool pdl = use_pdl(*d, shape->T);
-
-  LayoutParams p;
-  p.topk_idx = topk_idx;
-  p.T = shape->T;
-  p.k = shape->k;
-  p.E = shape->E;
-  p.R = shape->R;
-  p.Tr = shape->T / shape->R;
-  p.Er = shape->E / shape->R;
-  p.tile_t = g.tile_t;
-  p.tiles_per_rank = g.tiles_per_rank;
-  p.nt = g.nt;
-  p.ncol = g.ncol;
-  p.colhist = static_cast<int32_t*>(workspace);
-  p.coltotal = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + g.colhist_bytes);
-  p.num_tokens_per_expert = handle->num_tokens_per_expert;
-  p.expert_offset = handle->expert_offset;
-  p.num_tokens_per_rank = handle->num_tokens_per_rank;
-  p.count_src_rank_expert = handle->count_src_rank_expert;
-  p.src_rank_expert_offset = handle->src_rank_expert_offset;
-  p.is_token_in_rank = handle->is_token_in_rank;
-  p.slot_of_pair = handle->slot_of_pair;
-  p.src_of_slot = handle->src_of_slot;
-  p.error_word = handle->error_word;
-
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (shape->max_tokens_per_rank > 0) {
-    const size_t smem = layout_padded_smem(p.Tr, shape->E, shape->R);
-    if (smem > 48 * 1024) {
-      // a function attribute belongs to the current context (a reset or a
-      // green context starts without it), so it is set before each launch
-      const void* fn = shape->R <= kPadClusterMax ? reinterpret_cast<const void*>(layout_padded_kernel<true>)
-                                                  : reinterpret_cast<const void*>(layout_padded_kernel<false>);
-      if ((st = cuda_status(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem)))) != EP_OK)
-        return st;
-    }
-    if (shape->R <= kPadClusterMax) {  // one cluster of R CTAs sums the totals itself
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(shape->R);
-      cfg.blockDim = dim3(kPadThreads);
-      cfg.dynamicSmemBytes = smem;
-      cfg.stream = s;
-      cudaLaunchAttribute attr[2];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = shape->R;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = pdl_attribute(attr, 1, pdl);
-      if ((st = cuda_status(cudaLaunchKernelEx(&cfg, layout_padded_kernel<true>, p, shape->max_tokens_per_rank))) !=
-          EP_OK)
-        return st;
-      return finish(handle, s);
-    }
-    if ((st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_expert, 0, shape->E * 4, s))) != EP_OK ||
-        (st = cuda_status(cudaMemsetAsync(handle->num_tokens_per_rank, 0, shape->R * 4, s))) != EP_OK)
-      return st;
-    launch(pdl, layout_padded_kernel<false>, shape->R, kPadThreads, smem, s, p, shape->max_tokens_per_rank);
-    return finish(handle, s);
-  }
-  if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
-    launch(pdl, layout_small_kernel, kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R),
-        s, p);
-    return finish(handle, s);
-  }
-  if (g.nt > 0) {
-    const size_t smem = static_cast<size_t>(g.ncol) * 4 + static_cast<size_t>(g.tile_t) * shape->R;
-    launch(pdl, layout_count_kernel, g.nt, kLayoutThreads, smem, s, p);
-  }
-  launch(pdl, layout_scan_kernel, g.ncol, kLayoutThreads, 0, s, p);
-  const size_t smem_assign = static_cast<size_t>(shape->E + 1 + kLayoutWarps * shape->E) * 4;
-  launch(pdl, layout_assign_kernel, g.nt > 0 ? g.nt : 1, kLayoutThreads, smem_assign, s, p);
+  if ((st = enqueue_layout(shape, topk_idx, handle, workspace, g, use_pdl(*d, shape->T), false, s)) != EP_OK)
+    return st;
   return finish(handle, s);
 }
 
 int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weights, const ep_handle_t* handle,
                 void* recv_x, float* recv_scale, float* recv_weight, ep_stream_t stream) {
-  int st = check_shape(shape);
+  int st = check_dispatch_args(shape, x, topk_weights, handle, recv_x, recv_scale, recv_weight);
   if (st != EP_OK) return st;
-  if ((st = check_handle(shape, handle)) != EP_OK) return st;
-  const int64_t T = shape->T, P = T * shape->k;
-  if (!rows_ok(x, T) || !rows_ok(recv_x, P) || !f32_ok(topk_weights, P)) return EP_ERR_INVALID_ARG;
-  if (shape->use_fp8 && !f32_ok(recv_scale, P)) return EP_ERR_INVALID_ARG;
-  if (recv_weight != nullptr && !aligned(recv_weight, 4)) return EP_ERR_INVALID_ARG;
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
-  const bool pdl = use_pdl(*d, T);
-  if (T == 0) return EP_OK;
-  const MoveParams p = move_params(shape, handle, topk_weights, pdl);
+  if (shape->T == 0) return EP_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t units = T * p.chunks;
-  if (p.chunks >= kTmaMinChunks && p.chunks <= kTmaMaxChunks) {
-    const bool fp8 = shape->use_fp8 != 0;
-    const int threads = p.chunks * kWarp;
-    const size_t smem = tma_smem_layout(shape->H, fp8).total;
-    const void* fn = fp8 ? reinterpret_cast<const void*>(dispatch_tma_kernel<true>)
-                         : reinterpret_cast<const void*>(dispatch_tma_kernel<false>);
-    int occ;
-    {
-      std::lock_guard<std::mutex> lock(g_dev_mu);
-      int& cached = const_cast<DeviceInfo*>(d)->occ_tma[fp8][p.chunks];
-      if (cached == 0) cached = occupancy(fn, threads, smem);
-      occ = cached;
-    }
-    const int grid = tma_dispatch_grid(*d, shape, T, occ);
-    if (fp8)
-      launch(pdl, dispatch_tma_kernel<true>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x,
-          recv_scale, recv_weight);
-    else
-      launch(pdl, dispatch_tma_kernel<false>, grid, threads, smem, s, p, static_cast<const uint16_t*>(x), recv_x,
-          nullptr, recv_weight);
-  } else if (shape->use_fp8) {
-    launch(pdl, dispatch_kernel<true>, movement_grid(*d, shape, d->occ_disp_fp8, units), kMoveThreads, 0, s, p,
-        static_cast<const uint16_t*>(x), recv_x, recv_scale, recv_weight);
-  } else {
-    launch(pdl, dispatch_kernel<false>, movement_grid(*d, shape, d->occ_disp_bf16, units), kMoveThreads, 0, s, p,
-        static_cast<const uint16_t*>(x), recv_x, nullptr, recv_weight);
-  }
+  enqueue_dispatch(shape, x, topk_weights, handle, recv_x, recv_scale, recv_weight, d, use_pdl(*d, shape->T), false,
+                   s);
+  return finish(handle, s);
+}
+
+int ep_dispatch_with_layout(const ep_shape_t* shape, const int64_t* topk_idx, const void* x,
+                            const float* topk_weights, const ep_handle_t* handle, void* workspace,
+                            size_t workspace_bytes, void* recv_x, float* recv_scale, float* recv_weight,
+                            ep_stream_t stream) {
+  int st = ep_internal_check_layout_args(shape, topk_idx, handle);
+  if (st != EP_OK) return st;
+  if ((st = check_dispatch_args(shape, x, topk_weights, handle, recv_x, recv_scale, recv_weight)) != EP_OK) return st;
+  const LayoutGeometry g = layout_geometry(shape);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < g.total_bytes)
+    return EP_ERR_INVALID_ARG;
+  const DeviceInfo* d = nullptr;
+  if ((st = device_info(&d)) != EP_OK) return st;
+  const bool pdl = use_pdl(*d, shape->T);
+  const bool early = pdl && shape->T > 0 && tma_dispatch_applies(shape);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = enqueue_layout(shape, topk_idx, handle, workspace, g, pdl, early, s)) != EP_OK) return st;
+  if ((st = cuda_status(cudaGetLastError())) != EP_OK) return st;
+  if (shape->T > 0)
+    enqueue_dispatch(shape, x, topk_weights, handle, recv_x, recv_scale, recv_weight, d, pdl, early, s);
   return finish(handle, s);
 }
 

@@ -51,7 +51,24 @@ struct LayoutParams {
   int32_t* slot_of_pair;
   int32_t* src_of_slot;
   int32_t* error_word;
+  // 0: the kernel lets the next one on the stream be scheduled at its start.
+  // 1: only after its own programmatic-launch wait, so that the next kernel
+  // is scheduled only once every kernel before this one has completed (set on
+  // the last layout kernel of the fused layout + dispatch call, whose
+  // dispatch reads x before its own wait).
+  int late_trigger;
 };
+
+// The programmatic-launch prologue of every layout kernel: trigger, an
+// optional L2 prefetch of what the kernel reads first, wait (and the late
+// trigger described above).
+__device__ __forceinline__ void layout_trigger_early(const LayoutParams& p) {
+  if (!p.late_trigger) pdl_allow_next();
+}
+__device__ __forceinline__ void layout_wait(const LayoutParams& p) {
+  pdl_wait_prev();
+  if (p.late_trigger) pdl_allow_next();
+}
 
 __device__ __forceinline__ void tile_range(const LayoutParams& p, int tile, int& t0, int& t1) {
   const int r = tile / p.tiles_per_rank;
@@ -79,9 +96,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutPara
   bool bad = false;
   const int lane = threadIdx.x & (kWarp - 1);
   const int64_t* idx = p.topk_idx + static_cast<int64_t>(t0) * p.k;
-  pdl_allow_next();
+  layout_trigger_early(p);
   prefetch_l2(idx, static_cast<int64_t>(npairs) * 8, threadIdx.x, blockDim.x);
-  pdl_wait_prev();
+  layout_wait(p);
   // a tile holds at most kTilePairs pairs: every thread loads its (up to)
   // kPairsPerThread expert ids first, then counts them
   int e[kPairsPerThread];
@@ -162,8 +179,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scan_kernel(LayoutParam
   __shared__ int32_t scratch[kWarp];
   const int c = blockIdx.x;
   int32_t* col = p.colhist + static_cast<int64_t>(c) * p.nt;
-  pdl_allow_next();
-  pdl_wait_prev();
+  layout_trigger_early(p);
+  layout_wait(p);
   const int32_t total = block_exclusive_scan(col, p.nt, scratch);
   if (threadIdx.x == 0) p.coltotal[c] = total;
   if (c < p.E) {
@@ -201,8 +218,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
   const int my_lo = warp * S, my_hi = min(my_lo + S, npairs);
   int ereg[kMaxChunksPerWarp];
   bool bad = false;  // already reported by layout_count_kernel
-  pdl_allow_next();
-  pdl_wait_prev();
+  layout_trigger_early(p);
+  layout_wait(p);
 #pragma unroll
   for (int c = 0; c < kMaxChunksPerWarp; ++c) {
     const int i = my_lo + c * kWarp + lane;
@@ -342,9 +359,9 @@ layout_small_kernel(LayoutParams p) {
 
   bool bad = false;
   int ereg[kSmallChunks];
-  pdl_allow_next();
+  layout_trigger_early(p);
   prefetch_l2(p.topk_idx + pair0, static_cast<int64_t>(npairs) * 8, threadIdx.x, blockDim.x);
-  pdl_wait_prev();
+  layout_wait(p);
 #pragma unroll
   for (int q = 0; q < kSmallChunks; ++q) {
     const int i = my_lo + q * kWarp + lane;
@@ -525,9 +542,9 @@ __global__ void __launch_bounds__(kPadThreads) layout_padded_kernel(LayoutParams
 
   bool bad = false, over = false;
   int ereg[kPadChunks];
-  pdl_allow_next();
+  layout_trigger_early(p);
   prefetch_l2(p.topk_idx + pair0, static_cast<int64_t>(npairs) * 8, threadIdx.x, blockDim.x);
-  pdl_wait_prev();
+  layout_wait(p);
 #pragma unroll
   for (int q = 0; q < kPadChunks; ++q) {
     const int i = my_lo + q * kWarp + lane;

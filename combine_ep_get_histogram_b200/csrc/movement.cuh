@@ -197,24 +197,27 @@ constexpr int kTmaMaxChunks = 16;
 struct TmaSmemLayout {
   int row_bytes;   // payload row bytes, rounded up to 128
   int stages;      // payload row stages (2..3): as many as fit in kTmaRowBudget
-  int off_slot;    // int32 [2][kMaxK]
-  int off_w;       // float [2][kMaxK]
-  int off_scale;   // float [2][G]
+  int nbuf;        // slot / weight / scale buffers: 2, or one per row stage (early form)
+  int off_slot;    // int32 [nbuf][kMaxK]
+  int off_w;       // float [nbuf][kMaxK]
+  int off_scale;   // float [nbuf][G]
   int total;
 };
 
 constexpr int kTmaRowBudget = 40 * 1024;
+constexpr int kTmaMaxStages = 3;
 
-__host__ __device__ inline TmaSmemLayout tma_smem_layout(int H, bool fp8) {
+__host__ __device__ inline TmaSmemLayout tma_smem_layout(int H, bool fp8, bool early = false) {
   TmaSmemLayout L;
   const int row = fp8 ? H : 2 * H;
   L.row_bytes = (row + 127) / 128 * 128;
   L.stages = kTmaRowBudget / L.row_bytes;
-  L.stages = L.stages < 2 ? 2 : (L.stages > 3 ? 3 : L.stages);
+  L.stages = L.stages < 2 ? 2 : (L.stages > kTmaMaxStages ? kTmaMaxStages : L.stages);
+  L.nbuf = early ? L.stages : 2;
   L.off_slot = L.stages * L.row_bytes;
-  L.off_w = L.off_slot + 2 * kMaxK * 4;
-  L.off_scale = L.off_w + 2 * kMaxK * 4;
-  L.total = L.off_scale + (fp8 ? 2 * (H / kGroup) * 4 : 0);
+  L.off_w = L.off_slot + L.nbuf * kMaxK * 4;
+  L.off_scale = L.off_w + L.nbuf * kMaxK * 4;
+  L.total = L.off_scale + (fp8 ? L.nbuf * (H / kGroup) * 4 : 0);
   return L;
 }
 
@@ -230,12 +233,42 @@ __device__ __forceinline__ void bulk_store_row(void* gdst, uint32_t ssrc, int by
                :: "l"(gdst), "r"(ssrc), "r"(bytes) : "memory");
 }
 
+// One token's x chunk, quantised (FP8) or copied (BF16) into its row stage,
+// with its scales into sscale.
 template <bool FP8>
+__device__ __forceinline__ void tma_stage_row(uint8_t* row, float* sscale, const uint4& v0, const uint4& v1, int h0,
+                                              int h1, bool a0, bool a1, int lane) {
+  if constexpr (FP8) {
+    float sc0, sc1;
+    const uint2 q0 = quantize_piece(v0, sc0);
+    const uint2 q1 = quantize_piece(v1, sc1);
+    const bool scale_lane = (lane & (kLanesPerGroup - 1)) == 0;
+    if (a0) {
+      *reinterpret_cast<uint2*>(row + h0) = q0;
+      if (scale_lane) sscale[h0 / kGroup] = sc0;
+    }
+    if (a1) {
+      *reinterpret_cast<uint2*>(row + h1) = q1;
+      if (scale_lane) sscale[h1 / kGroup] = sc1;
+    }
+  } else {
+    if (a0) *reinterpret_cast<uint4*>(row + 2 * h0) = v0;
+    if (a1) *reinterpret_cast<uint4*>(row + 2 * h1) = v1;
+  }
+}
+
+// EARLY (the fused layout + dispatch call under programmatic launch): the
+// kernel before this one is the call's own layout, which lets this kernel be
+// scheduled only after its own wait, so every kernel before the call has
+// completed and x is final; the layout does not write x.  Each CTA then loads
+// and quantises its first tokens, one per row stage, before waiting for the
+// layout, and sends them once their slots are known.
+template <bool FP8, bool EARLY>
 __global__ void __launch_bounds__(kTmaMaxChunks * kWarp, 3)
 dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restrict__ recv_x,
                     float* __restrict__ recv_scale, float* __restrict__ recv_weight) {
   extern __shared__ __align__(128) uint8_t tma_smem[];
-  const TmaSmemLayout L = tma_smem_layout(p.H, FP8);
+  const TmaSmemLayout L = tma_smem_layout(p.H, FP8, EARLY);
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
   const int h0 = piece_channel(warp, lane), h1 = h0 + kHalfChunk;  // one chunk per warp
   const bool a0 = h0 < p.H, a1 = h1 < p.H;
@@ -243,17 +276,79 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
 
   uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
   int t = blockIdx.x;
+  int it0 = 0;
   // no prefetch in this prologue: its code cost the kernel a register spill
   // and 2-3 % at full batch
   if (p.pdl) pdl_allow_next();
-  if (p.pdl) pdl_wait_prev();
+  if constexpr (EARLY) {
+    int n_pre = 0;  // this CTA's tokens staged before the wait (CTA-uniform)
+    while (n_pre < L.stages && t + n_pre * static_cast<int>(gridDim.x) < p.T) ++n_pre;
+    if (n_pre > 0) {
+      const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
+      if (a0) v0 = ld_ro_v4(xr + h0);
+      if (a1) v1 = ld_ro_v4(xr + h1);
+    }
+    for (int i = 0; i < n_pre; ++i) {
+      uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+      if (i + 1 < n_pre) {
+        const uint16_t* xr = x + static_cast<int64_t>(t + (i + 1) * static_cast<int>(gridDim.x)) * p.H;
+        if (a0) n0 = ld_ro_v4(xr + h0);
+        if (a1) n1 = ld_ro_v4(xr + h1);
+      }
+      tma_stage_row<FP8>(tma_smem + i * L.row_bytes,
+                         reinterpret_cast<float*>(tma_smem + L.off_scale) + i * p.G, v0, v1, h0, h1, a0, a1, lane);
+      v0 = n0;
+      v1 = n1;
+    }
+    if (p.pdl) pdl_wait_prev();
+    if (n_pre > 0) {
+      // warp i reads the slots and gate weights of staged token i
+      if (warp < n_pre && lane < p.k) {
+        const int64_t pr = static_cast<int64_t>(t + warp * static_cast<int>(gridDim.x)) * p.k + lane;
+        reinterpret_cast<int32_t*>(tma_smem + L.off_slot)[warp * kMaxK + lane] = p.slot_of_pair[pr];
+        reinterpret_cast<float*>(tma_smem + L.off_w)[warp * kMaxK + lane] = p.topk_weights[pr];
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncthreads();
+      const int32_t* sslot = reinterpret_cast<const int32_t*>(tma_smem + L.off_slot);
+      if (threadIdx.x == 0) {
+        for (int i = 0; i < n_pre; ++i) {  // one bulk group per token, as in the loop below
+          const uint32_t src = static_cast<uint32_t>(__cvta_generic_to_shared(tma_smem + i * L.row_bytes));
+          for (int j = 0; j < p.k; ++j) {
+            const int s = sslot[i * kMaxK + j];
+            if (s >= 0) bulk_store_row(static_cast<uint8_t*>(recv_x) + static_cast<int64_t>(s) * row_bytes, src,
+                                       row_bytes);
+          }
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+      }
+      if constexpr (FP8) {
+        const float* sscale = reinterpret_cast<const float*>(tma_smem + L.off_scale);
+        for (int i = threadIdx.x; i < n_pre * p.k * p.G; i += blockDim.x) {
+          const int tj = i / p.G, g = i - tj * p.G;  // tj = token * k + j
+          const int s = sslot[(tj / p.k) * kMaxK + tj % p.k];
+          if (s >= 0) recv_scale[static_cast<int64_t>(s) * p.G + g] = sscale[(tj / p.k) * p.G + g];
+        }
+      }
+      if (recv_weight != nullptr && threadIdx.x < n_pre * p.k) {
+        const int i = threadIdx.x / p.k, j = threadIdx.x - i * p.k;
+        const int s = sslot[i * kMaxK + j];
+        if (s >= 0) recv_weight[s] = reinterpret_cast<const float*>(tma_smem + L.off_w)[i * kMaxK + j];
+      }
+    }
+    it0 = n_pre;
+    t += n_pre * static_cast<int>(gridDim.x);
+    v0 = v1 = make_uint4(0, 0, 0, 0);
+  } else {
+    if (p.pdl) pdl_wait_prev();
+  }
   if (t < p.T) {
     const uint16_t* xr = x + static_cast<int64_t>(t) * p.H;
     if (a0) v0 = ld_ro_v4(xr + h0);
     if (a1) v1 = ld_ro_v4(xr + h1);
   }
-  for (int it = 0; t < p.T; ++it, t += gridDim.x) {
-    const int stage = it & 1;
+  for (int it = it0; t < p.T; ++it, t += gridDim.x) {
+    const int stage = EARLY ? it % L.nbuf : (it & 1);
     uint8_t* row = tma_smem + (it % L.stages) * L.row_bytes;
     int32_t* sslot = reinterpret_cast<int32_t*>(tma_smem + L.off_slot) + stage * kMaxK;
     float* sw = reinterpret_cast<float*>(tma_smem + L.off_w) + stage * kMaxK;
@@ -272,23 +367,7 @@ dispatch_tma_kernel(MoveParams p, const uint16_t* __restrict__ x, void* __restri
     if (threadIdx.x == 0) bulk_wait_read_all_but(L.stages - 1);
     if (it > 0) __syncthreads();
 
-    if constexpr (FP8) {
-      float sc0, sc1;
-      const uint2 q0 = quantize_piece(v0, sc0);
-      const uint2 q1 = quantize_piece(v1, sc1);
-      const bool scale_lane = (lane & (kLanesPerGroup - 1)) == 0;
-      if (a0) {
-        *reinterpret_cast<uint2*>(row + h0) = q0;
-        if (scale_lane) sscale[h0 / kGroup] = sc0;
-      }
-      if (a1) {
-        *reinterpret_cast<uint2*>(row + h1) = q1;
-        if (scale_lane) sscale[h1 / kGroup] = sc1;
-      }
-    } else {
-      if (a0) *reinterpret_cast<uint4*>(row + 2 * h0) = v0;
-      if (a1) *reinterpret_cast<uint4*>(row + 2 * h1) = v1;
-    }
+    tma_stage_row<FP8>(row, sscale, v0, v1, h0, h1, a0, a1, lane);
     // the slots and weights after the quantisation: read before it, their
     // load held every warp at a barrier (decode dispatch 18.4 -> 16.9 us)
     if (warp == 0 && lane < p.k) {

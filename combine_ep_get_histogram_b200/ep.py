@@ -28,6 +28,7 @@ HANDLE_FIELDS = ("num_tokens_per_expert", "expert_offset", "num_tokens_per_rank"
                  "slot_of_pair", "src_of_slot", "error_word")
 
 EXPORTED = ("ep_handle_sizes", "ep_workspace_size", "ep_get_dispatch_layout", "ep_dispatch",
+            "ep_dispatch_with_layout",
             "ep_combine", "ep_combine_backward", "ep_dispatch_backward", "ep_get_error",
             "ep_status_string", "ep_last_cuda_error", "ep_get_dispatch_layout_noalloc",
             "ep_noalloc_scratch_bytes", "ep_route_group_limited", "ep_dispatch_peers", "ep_combine_peers",
@@ -80,6 +81,7 @@ def _lib():
             "ep_workspace_size": (ctypes.c_size_t, [shp]),
             "ep_get_dispatch_layout": (ctypes.c_int, [shp, vp, hp, vp, ctypes.c_size_t, vp]),
             "ep_dispatch": (ctypes.c_int, [shp, vp, vp, hp, vp, vp, vp, vp]),
+            "ep_dispatch_with_layout": (ctypes.c_int, [shp, vp, vp, vp, hp, vp, ctypes.c_size_t, vp, vp, vp, vp]),
             "ep_combine": (ctypes.c_int, [shp, vp, vp, hp, vp, vp]),
             "ep_combine_backward": (ctypes.c_int, [shp, vp, vp, vp, hp, vp, vp, vp]),
             "ep_dispatch_backward": (ctypes.c_int, [shp, vp, hp, vp, vp]),
@@ -208,6 +210,16 @@ def ep_dispatch(shape: ep_shape_t, x, topk_weights, handle: Handle, recv_x, recv
     st = _lib().ep_dispatch(ctypes.byref(shape), _ptr(x), _ptr(topk_weights), ctypes.byref(handle.c),
                             _ptr(recv_x), _ptr(recv_scale), _ptr(recv_weight), _stream(stream))
     return _check(st, "ep_dispatch") if check else st
+
+
+def ep_dispatch_with_layout(shape: ep_shape_t, topk_idx, x, topk_weights, handle: Handle, ws, recv_x,
+                            recv_scale=None, recv_weight=None, stream=None, check=True) -> int:
+    """ep_get_dispatch_layout and ep_dispatch in one call (see ep.h)."""
+    nbytes = ws.numel() if hasattr(ws, "numel") else workspace_size(shape)
+    st = _lib().ep_dispatch_with_layout(ctypes.byref(shape), _ptr(topk_idx), _ptr(x), _ptr(topk_weights),
+                                        ctypes.byref(handle.c), _ptr(ws), nbytes, _ptr(recv_x), _ptr(recv_scale),
+                                        _ptr(recv_weight), _stream(stream))
+    return _check(st, "ep_dispatch_with_layout") if check else st
 
 
 def ep_combine(shape: ep_shape_t, y, topk_weights, handle: Handle, out, stream=None, check=True) -> int:

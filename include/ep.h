@@ -161,6 +161,25 @@ int ep_dispatch(const ep_shape_t* shape, const void* x, const float* topk_weight
                 const ep_handle_t* handle, void* recv_x, float* recv_scale,
                 float* recv_weight, ep_stream_t stream);
 
+/* Layout and dispatch in one call, as the pages' dispatch takes x and
+ * topk_idx together and returns the received tokens with the handle
+ * ("DeepEP：MoE 专家并行 EP 通信 kernel 编译与使用指南" (zhouruolin.cn),
+ * section 五 使用方法).  Arguments are those of ep_get_dispatch_layout and
+ * ep_dispatch; every check of both runs before anything is enqueued, and the
+ * results (handle, recv_x, recv_scale, recv_weight, error word) are those of
+ * ep_get_dispatch_layout followed by ep_dispatch on the same stream.
+ * Below 16 tokens per SM with programmatic dependent launch, when H is
+ * 1536 < H <= 8192 (the bulk-store dispatch), the last layout kernel lets the
+ * dispatch kernel be scheduled only after its own wait, i.e. once everything
+ * enqueued before this call has completed, and each dispatch CTA then loads
+ * and quantises its first x rows (one per shared-memory row stage) while
+ * the layout still runs, sending them once their slots are known (the
+ * layout writes only the handle and the workspace, never x). */
+int ep_dispatch_with_layout(const ep_shape_t* shape, const int64_t* topk_idx, const void* x,
+                            const float* topk_weights, const ep_handle_t* handle,
+                            void* workspace, size_t workspace_bytes, void* recv_x,
+                            float* recv_scale, float* recv_weight, ep_stream_t stream);
+
 /* Combine: y [P,H] bf16 (expert outputs in receive order), topk_weights
  * [T,k] fp32 -> out [T,H] bf16.  A token with no valid pair gets +0. */
 int ep_combine(const ep_shape_t* shape, const void* y, const float* topk_weights,

@@ -77,6 +77,8 @@ def test_bad_shapes_rejected_on_host(kw):
     fake = 1 << 20  # never dereferenced: validation fails first
     assert lib.ep_get_dispatch_layout(ctypes.byref(s), fake, ctypes.byref(h), fake, 1 << 20, None) == 1
     assert lib.ep_dispatch(ctypes.byref(s), fake, fake, ctypes.byref(h), fake, fake, None, None) == 1
+    assert lib.ep_dispatch_with_layout(ctypes.byref(s), fake, fake, fake, ctypes.byref(h), fake, 1 << 20, fake, fake,
+                                       None, None) == 1
     assert lib.ep_combine(ctypes.byref(s), fake, fake, ctypes.byref(h), fake, None) == 1
     assert lib.ep_combine_backward(ctypes.byref(s), fake, fake, fake, ctypes.byref(h), fake, fake, None) == 1
     assert lib.ep_dispatch_backward(ctypes.byref(s), fake, ctypes.byref(h), fake, None) == 1
@@ -107,6 +109,13 @@ def test_bad_pointers_rejected_on_host():
     assert lib.ep_dispatch(sref, good, good, href, good + 2, good, None, None) == 1
     assert lib.ep_dispatch(sref, good, good, href, good, None, None, None) == 1
     assert lib.ep_dispatch(sref, good, good + 2, href, good, good, None, None) == 1
+    # layout + dispatch in one call: every check of both before anything runs
+    fused = lib.ep_dispatch_with_layout
+    assert fused(sref, None, good, good, href, good, ws, good, good, None, None) == 1
+    assert fused(sref, good, good + 8, good, href, good, ws, good, good, None, None) == 1
+    assert fused(sref, good, good, good, href, good, ws - 1, good, good, None, None) == 1
+    assert fused(sref, good, good, good, href, good, ws, good, None, None, None) == 1
+    assert fused(sref, good, good, good, ctypes.byref(h2), good, ws, good, good, None, None) == 1
     assert lib.ep_combine(sref, good + 8, good, href, good, None) == 1
     assert lib.ep_combine(sref, good, good, href, None, None) == 1
     assert lib.ep_combine_backward(sref, good, good, good, href, good, None, None) == 1

@@ -124,3 +124,14 @@ def test_reshape_options():
     assert (w.E, w.n_groups, w.topk_groups, w.routing, w.k) == (160, 4, 2, "group", 8)
     w = bench.workload(argparse.Namespace(**dict(base, groups=8, topk_groups=8)))
     assert (w.E, w.n_groups, w.topk_groups) == (256, 8, 8)
+
+
+def test_fused_dispatch_step_calls_and_bytes():
+    import argparse
+    from combine_ep_get_histogram_b200 import workloads as wl
+    a = argparse.Namespace(route=False, fused_dispatch=True)
+    assert bench.step_calls(a) == bench.FUSED_CALLS
+    assert bench.step_calls(argparse.Namespace(route=True, fused_dispatch=True))[0] == "route"
+    assert bench.step_calls(argparse.Namespace(route=False)) == bench.CALLS
+    b = bench.call_bytes(wl.CONFIGS["decode"])
+    assert b["dispatch_with_layout"] == b["layout"] + b["dispatch"]
