@@ -51,6 +51,7 @@ struct DeviceInfo {
   int occ_route[6] = {};          // route_group_limited_kernel<1, 2, 4, 8, 16, 32>
   int occ_route_aligned[6] = {};  // route_aligned_kernel<1, 2, 4, 8, 16, 32>
   int occ_route_compact[6][5] = {};  // route_compact_kernel<2^i, 2^j>, filled on first use
+  int small_cluster = 0;             // cluster size of layout_small_kernel, chosen on first use
 };
 
 constexpr int kMaxDevices = 64;
@@ -62,6 +63,32 @@ int occupancy(const void* fn, int threads, size_t smem) {
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) != cudaSuccess) return 1;
   return n > 0 ? n : 1;
+}
+
+// Cluster size of the one-launch layout on this device: the wide (16-CTA,
+// non-portable) cluster when the device can hold one with the kernel's
+// largest shared memory, else the portable 8.  The non-portable size needs a
+// function attribute, which belongs to the current context, so the launch
+// sets it again every time.
+int small_cluster_size(const DeviceInfo* d) {
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  int& c = const_cast<DeviceInfo*>(d)->small_cluster;
+  if (c == 0) {
+    const char* env = std::getenv("EP_LAYOUT_CLUSTER");  // "8": keep the portable size
+    if (env != nullptr && std::strcmp(env, "8") == 0) return c = kClusterCtas;
+    const cudaError_t before = cudaPeekAtLastError();
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterCtasWide);
+    cfg.blockDim = dim3(kSmallThreads);
+    cfg.dynamicSmemBytes = kSmallMaxSmem;
+    const bool ok = cudaFuncSetAttribute(layout_small_kernel<kClusterCtasWide>,
+                                         cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+                    cudaOccupancyMaxActiveClusters(&n, layout_small_kernel<kClusterCtasWide>, &cfg) == cudaSuccess;
+    if (!ok && before == cudaSuccess) (void)cudaGetLastError();  // the query's own error only
+    c = ok && n > 0 ? kClusterCtasWide : kClusterCtas;
+  }
+  return c;
 }
 
 int device_info(const DeviceInfo** out) {
@@ -403,7 +430,7 @@ int peer_setup(const ep_shape_t* shape, int32_t rank, const int64_t* topk_idx, c
 // caller).  late: the last kernel lets the next one be scheduled only after
 // its own programmatic-launch wait (LayoutParams::late_trigger).
 int enqueue_layout(const ep_shape_t* shape, const int64_t* topk_idx, const ep_handle_t* handle, void* workspace,
-                   const LayoutGeometry& g, bool pdl, bool late, cudaStream_t s) {
+                   const LayoutGeometry& g, const DeviceInfo* d, bool pdl, bool late, cudaStream_t s) {
   int st = EP_OK;
   LayoutParams p;
   p.topk_idx = topk_idx;
@@ -463,8 +490,16 @@ int enqueue_layout(const ep_shape_t* shape, const int64_t* topk_idx, const ep_ha
     return EP_OK;
   }
   if (layout_small_fits(shape->T, shape->k, shape->E, shape->R)) {
-    launch(pdl, layout_small_kernel, kClusterCtas, kSmallThreads, layout_small_smem(shape->T, shape->E, shape->R),
-        s, p);
+    if (small_cluster_size(d) == kClusterCtasWide) {
+      if ((st = cuda_status(cudaFuncSetAttribute(layout_small_kernel<kClusterCtasWide>,
+                                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1))) != EP_OK)
+        return st;
+      launch(pdl, layout_small_kernel<kClusterCtasWide>, kClusterCtasWide, kSmallThreads,
+             layout_small_smem(shape->T, shape->E, shape->R, kClusterCtasWide), s, p);
+    } else {
+      launch(pdl, layout_small_kernel<kClusterCtas>, kClusterCtas, kSmallThreads,
+             layout_small_smem(shape->T, shape->E, shape->R, kClusterCtas), s, p);
+    }
     return EP_OK;
   }
   // only the last of the three kernels triggers late
@@ -572,7 +607,7 @@ int ep_get_dispatch_layout(const ep_shape_t* shape, const int64_t* topk_idx, con
   const DeviceInfo* d = nullptr;
   if ((st = device_info(&d)) != EP_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if ((st = enqueue_layout(shape, topk_idx, handle, workspace, g, use_pdl(*d, shape->T), false, s)) != EP_OK)
+  if ((st = enqueue_layout(shape, topk_idx, handle, workspace, g, d, use_pdl(*d, shape->T), false, s)) != EP_OK)
     return st;
   return finish(handle, s);
 }
@@ -605,7 +640,7 @@ int ep_dispatch_with_layout(const ep_shape_t* shape, const int64_t* topk_idx, co
   const bool pdl = use_pdl(*d, shape->T);
   const bool early = pdl && shape->T > 0 && tma_dispatch_applies(shape);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if ((st = enqueue_layout(shape, topk_idx, handle, workspace, g, pdl, early, s)) != EP_OK) return st;
+  if ((st = enqueue_layout(shape, topk_idx, handle, workspace, g, d, pdl, early, s)) != EP_OK) return st;
   if ((st = cuda_status(cudaGetLastError())) != EP_OK) return st;
   if (shape->T > 0)
     enqueue_dispatch(shape, x, topk_weights, handle, recv_x, recv_scale, recv_weight, d, pdl, early, s);

@@ -295,8 +295,9 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
 // ----------------------------------------- small problems, one CTA cluster
 //
 // Up to kSmallMaxPairs pairs (the decode shape, 8 ranks x 128 tokens x
-// top-8, is 8192) are handled by one cluster of kClusterCtas CTAs on as many
-// SMs, in one launch.  CTA c takes the tile of whole tokens
+// top-8, is 8192) are handled by one cluster of C CTAs, in one launch: 16
+// (a non-portable cluster size) where the device can hold such a cluster,
+// else the portable 8.  CTA c takes the tile of whole tokens
 // [c*T/C, (c+1)*T/C).  Phase 1, per CTA: per-warp expert histograms of the
 // tile's pairs (each warp owns a contiguous run of pairs), per-(source rank,
 // expert) counts and per-rank token counts (warp-aggregated shared-memory
@@ -309,7 +310,8 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutPar
 // final cluster barrier keeps every CTA's shared memory alive until the
 // others have read it.
 
-constexpr int kClusterCtas = 8;
+constexpr int kClusterCtas = 8;      // portable cluster size
+constexpr int kClusterCtasWide = 16; // non-portable: halves each CTA's pairs (decode layout 14.7 -> 14.4 us per call)
 constexpr int kSmallThreads = 512;
 constexpr int kSmallWarps = kSmallThreads / kWarp;
 constexpr int kSmallMaxPairs = 16384;
@@ -317,24 +319,32 @@ constexpr int kSmallMaxE = 256;
 constexpr int kSmallMaxR = 64;
 constexpr int kSmallMaxRE = 2048;
 constexpr int kSmallMaxTileFlags = 8192;  // tile tokens x R flag bytes
-// pairs per CTA <= (T/C + 1) * k <= kSmallMaxPairs / C + kMaxK
-constexpr int kSmallChunks = ((kSmallMaxPairs / kClusterCtas + kMaxK) / kSmallWarps + kWarp - 1) / kWarp + 1;
+// pair chunks per warp: pairs per CTA <= (T/C + 1) * k <= kSmallMaxPairs / C + kMaxK
+__host__ __device__ constexpr int small_chunks(int C) {
+  return ((kSmallMaxPairs / C + kMaxK) / kSmallWarps + kWarp - 1) / kWarp + 1;
+}
 
-__host__ __device__ inline int small_tile_tokens(int T) { return (T + kClusterCtas - 1) / kClusterCtas; }
+__host__ __device__ inline int small_tile_tokens(int T, int C) { return (T + C - 1) / C; }
 
+// The limits are those of the 8-CTA cluster, whose tiles are the larger.
 __host__ __device__ inline bool layout_small_fits(int T, int k, int E, int R) {
   return static_cast<int64_t>(T) * k <= kSmallMaxPairs && E <= kSmallMaxE && R <= kSmallMaxR &&
-         R * E <= kSmallMaxRE && static_cast<int64_t>(small_tile_tokens(T)) * R <= kSmallMaxTileFlags;
+         R * E <= kSmallMaxRE && static_cast<int64_t>(small_tile_tokens(T, kClusterCtas)) * R <= kSmallMaxTileFlags;
 }
 
 // shared memory, int32 words then flag bytes:
 //   hist[E] base[E] whist[W][E] eoff[E+1] cnt[R*E] rank_cnt[R] flags[tile tokens * R]
-__host__ __device__ inline int layout_small_smem(int T, int E, int R) {
-  return (2 * E + kSmallWarps * E + (E + 1) + R * E + R) * 4 + small_tile_tokens(T) * R;
+__host__ __device__ inline int layout_small_smem(int T, int E, int R, int C) {
+  return (2 * E + kSmallWarps * E + (E + 1) + R * E + R) * 4 + small_tile_tokens(T, C) * R;
 }
+// the largest of the above over every shape layout_small_fits admits (36 KB)
+constexpr int kSmallMaxSmem =
+    (2 * kSmallMaxE + kSmallWarps * kSmallMaxE + (kSmallMaxE + 1) + kSmallMaxRE + kSmallMaxR) * 4 + kSmallMaxTileFlags;
 
-__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kSmallThreads)
+template <int C>
+__global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(kSmallThreads)
 layout_small_kernel(LayoutParams p) {
+  constexpr int kSmallChunks = small_chunks(C);
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ int32_t smem[];
@@ -348,8 +358,8 @@ layout_small_kernel(LayoutParams p) {
   __shared__ int32_t scratch[kWarp];
   const int c = static_cast<int>(cluster.block_rank());
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x / kWarp;
-  const int t0 = static_cast<int>(static_cast<int64_t>(c) * p.T / kClusterCtas);
-  const int t1 = static_cast<int>(static_cast<int64_t>(c + 1) * p.T / kClusterCtas);
+  const int t0 = static_cast<int>(static_cast<int64_t>(c) * p.T / C);
+  const int t1 = static_cast<int>(static_cast<int64_t>(c + 1) * p.T / C);
   const int ntok = t1 - t0;
   const int npairs = ntok * p.k;
   const int64_t pair0 = static_cast<int64_t>(t0) * p.k;
@@ -415,7 +425,7 @@ layout_small_kernel(LayoutParams p) {
   for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
     int32_t tot = 0, before = 0;
 #pragma unroll
-    for (int r = 0; r < kClusterCtas; ++r) {
+    for (int r = 0; r < C; ++r) {
       const int32_t n = cluster.map_shared_rank(hist, r)[e];
       before += r < c ? n : 0;
       tot += n;
@@ -464,7 +474,7 @@ layout_small_kernel(LayoutParams p) {
     for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
       int32_t n = 0;
 #pragma unroll
-      for (int q = 0; q < kClusterCtas; ++q) n += cluster.map_shared_rank(rank_cnt, q)[r];
+      for (int q = 0; q < C; ++q) n += cluster.map_shared_rank(rank_cnt, q)[r];
       p.num_tokens_per_rank[r] = n;
     }
   }
@@ -474,12 +484,12 @@ layout_small_kernel(LayoutParams p) {
   // ranks for the offsets.  whist is free again after the ranking loop.
   __syncthreads();
   int32_t* tot_re = whist;  // [R][e_hi - e_lo]
-  const int e_lo = c * p.E / kClusterCtas, e_hi = (c + 1) * p.E / kClusterCtas, ne = e_hi - e_lo;
+  const int e_lo = c * p.E / C, e_hi = (c + 1) * p.E / C, ne = e_hi - e_lo;
   for (int i = threadIdx.x; i < p.R * ne; i += blockDim.x) {
     const int r = i / ne, e = e_lo + (i - r * ne);
     int32_t m = 0;
 #pragma unroll
-    for (int q = 0; q < kClusterCtas; ++q) m += cluster.map_shared_rank(cnt, q)[r * p.E + e];
+    for (int q = 0; q < C; ++q) m += cluster.map_shared_rank(cnt, q)[r * p.E + e];
     tot_re[i] = m;
     p.count_src_rank_expert[r * p.E + e] = m;
   }
@@ -492,7 +502,7 @@ layout_small_kernel(LayoutParams p) {
     }
   }
   const int P = p.T * p.k;
-  for (int i = p_eff + c * blockDim.x + threadIdx.x; i < P; i += kClusterCtas * blockDim.x) p.src_of_slot[i] = -1;
+  for (int i = p_eff + c * blockDim.x + threadIdx.x; i < P; i += C * blockDim.x) p.src_of_slot[i] = -1;
   if (bad) atomicOr(p.error_word, 1);
   cluster.sync();  // keep this CTA's shared memory until the others are done reading it
 }

@@ -58,7 +58,13 @@
  *    launched with programmatic dependent launch (EP_PDL=0 turns it off): a
  *    kernel may become resident while the previous kernel on the stream
  *    finishes, but it reads and writes no global memory before that kernel
- *    has completed, so stream order is kept for any predecessor.
+ *    has completed, so stream order is kept for any predecessor.  (One
+ *    exception inside a call: ep_dispatch_with_layout's dispatch reads x while
+ *    the call's own layout still runs, which never writes x; everything
+ *    before the call has completed by then.)
+ *  - The one-launch layout (up to 16384 pairs) runs as one thread-block
+ *    cluster of 16 CTAs, a non-portable cluster size, where the device can
+ *    hold one, else 8; EP_LAYOUT_CLUSTER=8 keeps it at 8.
  *  - bf16 arrays are uint16 bit patterns; rows of bf16 / fp8 arrays must start
  *    on 16-byte boundaries (H % 8 == 0 and 16-byte aligned base pointers).
  *  - Return value: EP_OK or an ep_status_t code.  Argument errors are found

@@ -221,3 +221,19 @@ def test_small_batch_gathers(cuda_device, T, H, k, masked, num_sms):
     E, R = 32, 4
     idx = random_idx(T, k, E, seed=T + k, masked=masked, distinct=masked == 0.0)
     run_and_compare(cuda_device, T, H, k, E, R, False, idx, num_sms=num_sms)
+
+
+def test_portable_cluster_layout():
+    """The one-launch layout with the portable 8-CTA cluster (EP_LAYOUT_CLUSTER=8;
+    a B200 otherwise takes the 16-CTA one): the shape tests again, in a
+    process of their own."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, EP_LAYOUT_CLUSTER="8")
+    here = os.path.dirname(os.path.abspath(__file__))
+    files = [os.path.join(here, f) for f in ("test_gpu_edge.py", "test_gpu_fused.py")]
+    pick = "test_shapes or test_masked_and_duplicate or test_fused_matches"
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
+                        "-k", pick] + files, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
