@@ -41,6 +41,10 @@ def test_bench_line_has_the_contract_keys(cuda_device):
     assert d["gpu_launches"] == 5 * 4
     for call in ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward"):
         assert d["per_call"][call]["us"] > 0
+        # tiny is timed cold per call, beside a same-size copy timed the same way
+        copy = d["per_call"][call]["same_size_copy"]
+        assert copy["us"] > 0 and copy["GB_s"] > 0
+        assert abs(copy["frac_of_copy"] - copy["us"] / d["per_call"][call]["us"]) < 3e-3
     both = d["dispatch_incl_layout"]  # dispatch with its layout
     assert abs(both["us"] - d["per_call"]["layout"]["us"] - d["per_call"]["dispatch"]["us"]) < 0.02
     load = d["load"]  # load skew from the layout's counts: max over mean, at least 1
@@ -68,3 +72,18 @@ def test_bench_line_for_the_emulated_ranks(cuda_device):
     assert d["gpu_launches"] == (1 + 4 * 4) * 4
     for call in ("layout", "dispatch", "combine", "combine_backward", "dispatch_backward"):
         assert d["per_call"][call]["us"] > 0
+
+
+def test_bench_line_with_the_fused_dispatch(cuda_device):
+    """--fused-dispatch: the layout and the dispatch as one call, same kernels."""
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "tiny", "--fused-dispatch",
+                        "--steps", "4", "--warmup", "3", "--no-e2e", "--no-cpu-baseline"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["config"]["dispatch_call"].startswith("fused")
+    assert set(d["per_call"]) == {"dispatch_with_layout", "combine", "combine_backward", "dispatch_backward"}
+    assert d["gpu_launches"] == 5 * 4
+    assert d["value"] > 0
