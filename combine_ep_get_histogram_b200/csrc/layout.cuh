@@ -465,33 +465,36 @@ layout_small_kernel(LayoutParams p) {
     __syncwarp();
   }
 
-  // summaries, spread over the cluster
-  if (c == 0) {
-    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) {
-      p.expert_offset[e] = eoff[e];
-      if (e < p.E) p.num_tokens_per_expert[e] = eoff[e + 1] - eoff[e];
-    }
-    for (int r = threadIdx.x; r < p.R; r += blockDim.x) {
-      int32_t n = 0;
-#pragma unroll
-      for (int q = 0; q < C; ++q) n += cluster.map_shared_rank(rank_cnt, q)[r];
-      p.num_tokens_per_rank[r] = n;
-    }
+  // summaries, spread over the cluster: CTA c owns experts [e_lo, e_hi) and
+  // writes their offsets and counts (CTA C-1 also the end offset), and the
+  // token counts of destination ranks c, c + C, ...  One thread per (rank,
+  // owned expert) and one per owned destination rank gather the cluster's
+  // counts in a single round of distributed-shared-memory loads; then one
+  // thread per owned expert walks the ranks for the offsets.  whist is free
+  // again after the ranking loop.
+  const int e_lo = c * p.E / C, e_hi = (c + 1) * p.E / C, ne = e_hi - e_lo;
+  for (int e = e_lo + threadIdx.x; e < e_hi; e += blockDim.x) {
+    p.expert_offset[e] = eoff[e];
+    p.num_tokens_per_expert[e] = eoff[e + 1] - eoff[e];
   }
-  // per-(source rank, expert) totals: CTA c owns experts [e_lo, e_hi); one
-  // thread per (rank, owned expert) gathers the cluster's counts in one round
-  // of distributed-shared-memory loads, then one thread per expert walks the
-  // ranks for the offsets.  whist is free again after the ranking loop.
+  if (c == C - 1 && threadIdx.x == 0) p.expert_offset[p.E] = eoff[p.E];
   __syncthreads();
   int32_t* tot_re = whist;  // [R][e_hi - e_lo]
-  const int e_lo = c * p.E / C, e_hi = (c + 1) * p.E / C, ne = e_hi - e_lo;
-  for (int i = threadIdx.x; i < p.R * ne; i += blockDim.x) {
-    const int r = i / ne, e = e_lo + (i - r * ne);
+  const int nre = p.R * ne, nr = (p.R - c + C - 1) / C;
+  for (int i = threadIdx.x; i < nre + nr; i += blockDim.x) {
+    const bool re = i < nre;
+    const int r = re ? i / ne : c + C * (i - nre);
+    const int e = re ? e_lo + (i - r * ne) : 0;
+    int32_t* word = re ? cnt + r * p.E + e : rank_cnt + r;  // this CTA's copy; the others' at the same offset
     int32_t m = 0;
 #pragma unroll
-    for (int q = 0; q < C; ++q) m += cluster.map_shared_rank(cnt, q)[r * p.E + e];
-    tot_re[i] = m;
-    p.count_src_rank_expert[r * p.E + e] = m;
+    for (int q = 0; q < C; ++q) m += *cluster.map_shared_rank(word, q);
+    if (re) {
+      tot_re[i] = m;
+      p.count_src_rank_expert[r * p.E + e] = m;
+    } else {
+      p.num_tokens_per_rank[r] = m;
+    }
   }
   __syncthreads();
   for (int el = threadIdx.x; el < ne; el += blockDim.x) {
