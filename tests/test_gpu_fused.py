@@ -75,6 +75,8 @@ class Fused:
     (1024, 7168, 8, 256, 8, True, 0, 128),   # padded layout (one cluster) before the early dispatch
     (512, 2048, 4, 64, 16, True, 0, 40),     # padded layout with 16 ranks (atomics)
     (8, 4096, 4, 16, 4, True, 0, 0),         # fewer tokens than CTAs
+    (512, 8192, 4, 64, 8, False, 8, 0),      # BF16 at H = 8192: two row stages, then the loop (8-SM budget)
+    (512, 8192, 32, 64, 8, True, 0, 0),      # k = 32: every lane of a staging warp reads a slot
     (6144, 4096, 8, 128, 8, False, 0, 0),    # 41 tokens per SM: no programmatic launch, plain dispatch
     (256, 256, 4, 16, 4, True, 0, 0),        # H = 256: the warp-per-chunk dispatch
 ])
@@ -168,3 +170,27 @@ def test_fused_equals_the_two_calls(cuda_device):
     for n in LAYOUT_FIELDS:
         assert torch.equal(a.handle.tensors[n], b.handle.tensors[n]), n
     assert torch.equal(a.rx, b.rx) and torch.equal(a.rs, b.rs) and torch.equal(a.rw, b.rw)
+
+
+def test_fused_bad_index(cuda_device):
+    """An out-of-range expert id through the fused call: the pair is masked
+    and the error word reports it, as with the two separate calls."""
+    T, H, k, E, R = 256, 2048, 4, 16, 4
+    idx = _routing(T, k, E, seed=21)
+    idx[7, 2] = E + 5
+    wts = np.random.default_rng(22).uniform(0.05, 1.0, (T, k)).astype(np.float32)
+    x = wl.normal_bf16(T, H, 23, 1)
+    f = Fused(cuda_device, T, H, k, E, R, True)
+    f.call(to_dev(idx, cuda_device), to_dev(x, cuda_device), to_dev(wts, cuda_device))
+    torch.cuda.synchronize()
+    ref = oracle.layout(idx, E, R)
+    assert ref["slot_of_pair"][7 * k + 2] == -1
+    counts = ep.handle_sizes(f.shape)
+    got = {n: f.handle.tensors[n].cpu().numpy()[: counts[n]] for n in LAYOUT_FIELDS}
+    assert_layout_equal(got, ref)
+    slots = ref["slot_of_pair"]
+    used = np.sort(slots[slots >= 0])
+    rx, rs, rw = oracle.dispatch(x, wts, slots, True)
+    assert_bits_equal("recv_x", f.rx.cpu().numpy()[used], rx[used])
+    assert_bits_equal("recv_scale", f.rs.cpu().numpy()[used].view(np.uint32), rs[used].view(np.uint32))
+    assert ep.ep_get_error(f.handle) == ep.ep.EP_ERR_BAD_INDEX
