@@ -111,13 +111,13 @@ typedef struct {
                       their grids is capped at num_sms x (CTAs of that kernel
                       resident per SM), so the caller's own kernels keep the
                       rest ("deepep-expert-parallel-communication-library",
-                      "deepep-expert-parallel-communication-library", section 二 SM 资源控制).  The
-                      hardware places a grid's CTAs on distinct SMs before it
-                      stacks them, so the CTAs land on num_sms SMs only when
-                      the stream belongs to an SM partition of that size (a
-                      CUDA green context).  The layout kernels (tens of
-                      microseconds) are not capped.  Results do not depend on
-                      the budget. */
+                      section 二 SM 资源控制).  The hardware places a grid's
+                      CTAs on distinct SMs before it stacks them, so the CTAs
+                      land on num_sms SMs only when the stream belongs to an
+                      SM partition of that size (a CUDA green context).  The
+                      layout kernels (microseconds; the one-launch layout is
+                      one cluster of 16 or 8 CTAs) are not capped.  Results
+                      do not depend on the budget. */
   int32_t max_tokens_per_rank; /* 0: dense receive layout (below).  M > 0:
                       the padded low-latency layout: E*R*M receive rows, one
                       block of M rows per (expert e, source rank r) at row
