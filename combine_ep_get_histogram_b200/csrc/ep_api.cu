@@ -67,9 +67,11 @@ int occupancy(const void* fn, int threads, size_t smem) {
 
 // Cluster size of the one-launch layout on this device: the wide (16-CTA,
 // non-portable) cluster when the device can hold one with the kernel's
-// largest shared memory, else the portable 8.  The non-portable size needs a
-// function attribute, which belongs to the current context, so the launch
-// sets it again every time.
+// largest shared memory, else the portable 8.  The choice is made once per
+// device, in the first context that runs the layout (EP_LAYOUT_CLUSTER=8
+// keeps the portable size for a context with fewer SMs).  The non-portable
+// size needs a function attribute, which belongs to the current context, so
+// the launch sets it again every time.
 int small_cluster_size(const DeviceInfo* d) {
   std::lock_guard<std::mutex> lock(g_dev_mu);
   int& c = const_cast<DeviceInfo*>(d)->small_cluster;
